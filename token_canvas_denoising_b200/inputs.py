@@ -1,0 +1,194 @@
+"""Seeded synthetic inputs for the canvas denoise path.
+
+This module only draws numbers: weights, prompt-prefix K/V, per-position
+inverse temperatures and canvas seeds. It holds none of the method's
+arithmetic, so both the CUDA path (tests, bench, smoke) and the fp64 oracle can
+be fed from it without sharing computation.
+
+Workloads follow the five synthetic configurations of the method's hot path
+(no trained weights or prompts exist here, so these stand in for them):
+
+  tiny       B1 C16  S32     d64   Hq2/Hk1  h32  V512     f32   T=8
+  canvas256  B1 C256 S1024   d2048 Hq16/Hk8 h128 V32768   bf16  T=48
+  vocab262k  B1 C256 S4096   d2816 Hq16/Hk8 h128 V262144  bf16  T=48, invT log-uniform [1/5, 1/0.05]
+  longctx    B4 C256 S32768  d2816 Hq16/Hk8 h128 V262144  bf16  T=48, prefix scale U[0.5, 2] per (request, head)
+  moe        vocab262k + MoE 128 experts + 1 shared, top-8, GeGLU intermediate 704
+
+Weights are N(0, std) with std = 1/sqrt(fan_in), fan_in being the contraction
+dimension of the matrix; the embedding table uses std 1 (a one-hot lookup reads
+one input). Prefix K/V are N(0, 1). Every tensor has its own Philox stream
+(numpy's Philox-4x64 keyed on (weight seed, tensor id)); bf16 tensors are drawn
+in float32 and rounded once to bf16 (round to nearest even) and are returned as
+uint16 bit patterns.
+"""
+from dataclasses import dataclass, field, replace
+import math
+
+import numpy as np
+
+# tensor ids of the per-tensor Philox streams
+_TID = {"embed": 1, "wq": 2, "wk": 3, "wv": 4, "wo": 5, "lm_head": 6,
+        "prefix_scale": 100, "inv_temp": 101, "w_router": 200}
+
+
+@dataclass(frozen=True)
+class Config:
+    name: str
+    B: int
+    C: int
+    S: tuple            # prefix length per request
+    d: int
+    Hq: int
+    Hk: int
+    h: int
+    V: int
+    dtype: str          # "f32" or "bf16"
+    max_steps: int
+    weight_seed: int
+    canvas_seeds: tuple
+    inv_temp: str = "one"          # "one" or "loguniform"
+    prefix_scale: bool = False     # per (request, kv head) scale U[0.5, 2]
+    n_experts: int = 0
+    top_k: int = 0
+    moe_inter: int = 0
+    n_shared: int = 0
+    stop_entropy: float = 0.05
+
+    @property
+    def M(self):
+        return self.B * self.C
+
+
+def _seeds(n, B):
+    return tuple(n * 100 + b for b in range(B))
+
+
+CONFIGS = {
+    "tiny": Config("tiny", 1, 16, (32,), 64, 2, 1, 32, 512, "f32", 8, 1001, (0,)),
+    "canvas256": Config("canvas256", 1, 256, (1024,), 2048, 16, 8, 128, 32768, "bf16",
+                        48, 1002, _seeds(2, 1)),
+    "vocab262k": Config("vocab262k", 1, 256, (4096,), 2816, 16, 8, 128, 262144, "bf16",
+                        48, 1003, _seeds(3, 1), inv_temp="loguniform"),
+    "longctx": Config("longctx", 4, 256, (32768,) * 4, 2816, 16, 8, 128, 262144, "bf16",
+                      48, 1004, _seeds(4, 4), prefix_scale=True),
+    "moe": Config("moe", 1, 256, (4096,), 2816, 16, 8, 128, 262144, "bf16", 48, 1005,
+                  _seeds(5, 1), inv_temp="loguniform", n_experts=128, top_k=8,
+                  moe_inter=704, n_shared=1),
+}
+CONFIG_ORDER = ["tiny", "canvas256", "vocab262k", "longctx", "moe"]
+
+
+def derive(cfg, **over):
+    """A copy of a configuration with some fields changed (smaller test cases)."""
+    if "B" in over and "canvas_seeds" not in over:
+        base = cfg.canvas_seeds[0] if cfg.canvas_seeds else 0
+        over["canvas_seeds"] = tuple(base + b for b in range(over["B"]))
+    if "B" in over and "S" not in over:
+        over["S"] = tuple(cfg.S[0] for _ in range(over["B"]))
+    return replace(cfg, **over)
+
+
+def _rng(seed, tid):
+    # one 128-bit integer key: numpy reads a list key through float64
+    return np.random.Generator(np.random.Philox(key=int(seed) | (int(tid) << 64)))
+
+
+def f32_to_bf16_bits(x):
+    """float32 -> bf16 bit patterns, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    return ((u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b):
+    return (np.asarray(b, np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def normal(seed, tid, shape, std, dtype, chunk_rows=8192):
+    """N(0, std) tensor of the given shape in storage dtype (uint16 bf16 bits or f32).
+
+    Drawn row-chunk by row-chunk from one Philox stream to bound host memory."""
+    rng = _rng(seed, tid)
+    shape = tuple(int(s) for s in shape)
+    rows = shape[0]
+    inner = int(np.prod(shape[1:])) if len(shape) > 1 else 1
+    out = np.empty((rows, inner), dtype=np.uint16 if dtype == "bf16" else np.float32)
+    for r0 in range(0, rows, chunk_rows):
+        r1 = min(rows, r0 + chunk_rows)
+        x = rng.standard_normal((r1 - r0, inner), dtype=np.float32)
+        x *= np.float32(std)
+        out[r0:r1] = f32_to_bf16_bits(x) if dtype == "bf16" else x
+    return out.reshape(shape)
+
+
+@dataclass
+class Workload:
+    cfg: Config
+    weights: dict                  # name -> numpy array (uint16 bf16 bits or float32)
+    prefix_k: list                 # per request [S_b, Hk, h]
+    prefix_v: list
+    inv_temp: np.ndarray           # float32 [B*C]
+    seeds: np.ndarray              # uint64 [B]
+    extra: dict = field(default_factory=dict)
+
+
+def make_workload(cfg, weight_overrides=None):
+    """Draw every input of a configuration. weight_overrides maps a tensor name
+    to an array that replaces the drawn one (used to inject known values)."""
+    c = cfg
+    dt = c.dtype
+    w = {}
+    ov = dict(weight_overrides or {})
+
+    def draw(name, shape, std, tid=None):
+        if name in ov:
+            w[name] = ov.pop(name)
+        else:
+            w[name] = normal(c.weight_seed, _TID[name] if tid is None else tid, shape, std, dt)
+
+    draw("embed", (c.V, c.d), 1.0)
+    draw("wq", (c.Hq * c.h, c.d), 1.0 / math.sqrt(c.d))
+    draw("wk", (c.Hk * c.h, c.d), 1.0 / math.sqrt(c.d))
+    draw("wv", (c.Hk * c.h, c.d), 1.0 / math.sqrt(c.d))
+    draw("wo", (c.d, c.Hq * c.h), 1.0 / math.sqrt(c.Hq * c.h))
+    draw("lm_head", (c.V, c.d), 1.0 / math.sqrt(c.d))
+    if c.n_experts:
+        ne = c.n_experts + c.n_shared
+        draw("w_router", (c.n_experts, c.d), 1.0 / math.sqrt(c.d))
+        for name, shape, std, base in (
+                ("w_gate", (c.moe_inter, c.d), 1.0 / math.sqrt(c.d), 1000),
+                ("w_up", (c.moe_inter, c.d), 1.0 / math.sqrt(c.d), 2000),
+                ("w_down", (c.d, c.moe_inter), 1.0 / math.sqrt(c.moe_inter), 3000)):
+            if name in ov:
+                w[name] = ov.pop(name)
+                continue
+            arr = np.empty((ne,) + shape, dtype=np.uint16 if dt == "bf16" else np.float32)
+            for e in range(ne):
+                arr[e] = normal(c.weight_seed, base + e, shape, std, dt)
+            w[name] = arr
+    if ov:
+        raise KeyError(f"unknown weight overrides: {sorted(ov)}")
+
+    scales = None
+    if c.prefix_scale:
+        scales = _rng(c.weight_seed, _TID["prefix_scale"]).uniform(
+            0.5, 2.0, size=(c.B, c.Hk)).astype(np.float32)
+    pk, pv = [], []
+    for b in range(c.B):
+        S = c.S[b]
+        for lst, tid in ((pk, 10 + 2 * b), (pv, 11 + 2 * b)):
+            rng = _rng(c.weight_seed, tid)
+            x = rng.standard_normal((S, c.Hk, c.h), dtype=np.float32)
+            if scales is not None:
+                x *= scales[b][None, :, None]
+            lst.append(f32_to_bf16_bits(x) if dt == "bf16" else x)
+
+    if c.inv_temp == "loguniform":
+        T = np.exp(_rng(c.weight_seed, _TID["inv_temp"]).uniform(
+            math.log(0.05), math.log(5.0), size=c.B * c.C))
+        inv_temp = (1.0 / T).astype(np.float32)
+    else:
+        inv_temp = np.ones(c.B * c.C, dtype=np.float32)
+    seeds = np.array(c.canvas_seeds, dtype=np.uint64)
+    return Workload(c, w, pk, pv, inv_temp, seeds,
+                    {"prefix_scale": scales})

@@ -1,0 +1,180 @@
+/*
+ * dg_canvas.h -- C ABI of libdgcanvas.so: the per-step denoise of a token
+ * canvas (DiffusionGemma-style block diffusion decoding) on one NVIDIA B200.
+ *
+ * What one denoise step computes, and where the method is described
+ * ("DiffusionGemma解析：扩散模型如何让LLM快5倍" = [P1],
+ *  "DiffusionGemma深度拆解：从逐字蹦到整块喷，LLM生成范式的结构性跃迁" = [P3],
+ *  "谷歌DiffusionGemma：并行生成与自纠的新突破" = [P4]):
+ *   1. embed the canvas tokens (a block of up to 256 positions; [P1] 整片并行去噪,
+ *      [P3] 架构解剖 diagram, [P4] 工作原理);
+ *   2. project Q and the canvas's own K/V, recomputed every step ([P3] 架构解剖 2);
+ *   3. bidirectional GQA attention of every canvas query over the cached prompt
+ *      K/V prefix plus the canvas K/V, no mask ([P1] 整片并行去噪 last paragraph,
+ *      [P3] 架构解剖 2 and diagram);
+ *   4. output projection with residual; optionally an MoE FFN with 128 experts,
+ *      top-8 routing and one shared expert ([P3] 架构解剖 3);
+ *   5. the LM head over the vocabulary fused with a per-position softmax
+ *      entropy and argmax; logits are never written to memory ([P1]
+ *      整片并行去噪: one distribution per position, lower entropy = more sure);
+ *   6. entropy-ordered freezing of the most certain unfrozen positions, each
+ *      taking its argmax token ([P1] 整片并行去噪, [P4] 工作原理);
+ *   7. re-noising every other unfrozen position with a fresh uniform token id
+ *      (unified-state noise, not [MASK]: [P3] 架构解剖 4, [P4] 工作原理), and an
+ *      adaptive stop within the step cap ([P1] 自适应停步机制: at most 48 steps).
+ *
+ * Conventions (apply to every entry point):
+ *   - All matrices are row-major; weights are stored [out][in], so both GEMM
+ *     operands are contiguous along the contraction dimension.
+ *   - "device" pointers are CUDA device memory on the current device; "host"
+ *     pointers are ordinary CPU memory. Caller-owned buffers are never freed by
+ *     the library. The library owns its workspace and the canvas state and
+ *     releases them in dg_canvas_destroy.
+ *   - Work is queued on the CUDA stream given to dg_canvas_init (NULL = the
+ *     legacy default stream) and is stream-ordered. Calls marked "synchronous"
+ *     wait for the stream.
+ *   - Errors are reported by status code only; nothing is thrown across the
+ *     ABI. Arguments are validated before any launch. Device-side checks
+ *     (token id out of range, NaN entropy, a bounded wait that gave up) set an
+ *     error word that the next synchronous call reports as
+ *     DG_ERR_DEVICE_CHECK / DG_ERR_TIMEOUT; kernels never trap.
+ *   - A context must not be used from two host threads at once.
+ *   - Shapes supported: canvas_len 1..256; storage dtype f32 (CUDA-core
+ *     kernels, head_dim 32..128 multiple of 32) or bf16 (tensor-core kernels,
+ *     head_dim 128, d_model a multiple of 64, vocab a multiple of 256,
+ *     n_q_heads a multiple of n_kv_heads).
+ */
+#ifndef DG_CANVAS_H
+#define DG_CANVAS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DG_ABI_VERSION 1
+
+typedef enum dg_status {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent shapes */
+  DG_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes/dtypes */
+  DG_ERR_OOM = 3,           /* workspace allocation failed (or over DG_WORKSPACE_LIMIT_MB) */
+  DG_ERR_CUDA = 4,          /* a CUDA runtime call failed; see dg_last_error() */
+  DG_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up */
+  DG_ERR_DEVICE_CHECK = 6   /* a device-side argument/data check failed */
+} dg_status;
+
+typedef enum dg_dtype { DG_F32 = 0, DG_BF16 = 1 } dg_dtype;
+
+/* Weights of the single-layer canvas denoiser. All pointers are device,
+ * caller-owned, in the storage dtype `dtype`, and must stay valid until
+ * dg_canvas_destroy. */
+typedef struct dg_model_desc {
+  int32_t d_model, n_q_heads, n_kv_heads, head_dim, vocab, dtype;
+  const void *embed;    /* [vocab][d_model]                       */
+  const void *wq;       /* [n_q_heads*head_dim][d_model]          */
+  const void *wk;       /* [n_kv_heads*head_dim][d_model]         */
+  const void *wv;       /* [n_kv_heads*head_dim][d_model]         */
+  const void *wo;       /* [d_model][n_q_heads*head_dim]          */
+  const void *lm_head;  /* [vocab][d_model]                       */
+  /* MoE FFN after attention; n_experts = 0 disables it. */
+  int32_t n_experts, top_k, moe_inter, n_shared;
+  const void *w_router; /* [n_experts][d_model]                   */
+  const void *w_gate;   /* [n_experts+n_shared][moe_inter][d_model] */
+  const void *w_up;     /* [n_experts+n_shared][moe_inter][d_model] */
+  const void *w_down;   /* [n_experts+n_shared][d_model][moe_inter] */
+} dg_model_desc;
+
+/* Freeze schedule and stop rule ([P1] 整片并行去噪, 自适应停步机制).
+ * At step t of a canvas with U unfrozen positions, k = ceil(U / (max_steps - t))
+ * positions freeze (all of them when max_steps - t <= 1). With adaptive_stop,
+ * the canvas stops once the smallest entropy among positions still unfrozen
+ * after freezing is below stop_entropy (nats); the rest then take their argmax. */
+typedef struct dg_schedule {
+  int32_t max_steps;     /* 1..1024; the pages' cap is 48 */
+  float stop_entropy;    /* nats; 0.05 in the reference configuration */
+  int32_t adaptive_stop; /* 0 = run every canvas to full freeze */
+  int32_t kind;          /* DG_SCHED_CEIL (only value) */
+} dg_schedule;
+#define DG_SCHED_CEIL 0
+
+/* Optional per-step outputs of dg_denoise_step (each device, may be NULL). */
+typedef struct dg_step_out {
+  float *ent;           /* [B*C] entropy of softmax(logits * inv_temp), nats   */
+  int32_t *argmax;      /* [B*C] argmax of the unscaled logits, lowest id on ties */
+  uint8_t *freeze_mask; /* [B*C] 1 where the position froze at this step        */
+  void *attn_out;       /* [B*C][n_q_heads*head_dim] attention output O (dtype) */
+  void *hidden;         /* [B*C][d_model] residual stream fed to the LM head   */
+} dg_step_out;
+
+/* Host-side copy of the decode state (all host arrays). */
+typedef struct dg_state {
+  int32_t *tokens;  /* [B*C] current canvas token ids                      */
+  uint8_t *frozen;  /* [B*C] 1 = frozen (never changes again)              */
+  int32_t *step;    /* [B]   steps completed by each canvas               */
+  uint64_t *seed;   /* [B]   Philox seed of each canvas                   */
+  uint8_t *done;    /* [B]   1 = canvas finished (stopped)                */
+} dg_state;
+
+typedef struct dg_ctx dg_ctx;
+
+/* Create a decode context and draw the initial canvases.
+ *   model       weights (see dg_model_desc); copied by value.
+ *   batch       B >= 1 independent canvases (requests).
+ *   canvas_len  C, 1..256 positions per canvas.
+ *   prefix_len  host [B]: cached prompt length S_b >= 0 of each request.
+ *   prefix_k/v  host arrays of B device pointers, each [S_b][n_kv_heads][head_dim]
+ *               in the storage dtype (NULL allowed when S_b = 0).
+ *   inv_temp    device [B*C] f32 per-position inverse temperature applied to the
+ *               logits before the entropy, or NULL for 1.
+ *   seeds       host [B] Philox seeds; canvas b position p starts at
+ *               draw(seeds[b], step 0, p, b).
+ *   cuda_stream cudaStream_t to queue all work on (NULL = default stream).
+ * Allocates the workspace (DG_ERR_OOM on failure). Returns DG_OK and *out. */
+dg_status dg_canvas_init(dg_ctx **out, const dg_model_desc *model, int32_t batch,
+                         int32_t canvas_len, const int32_t *prefix_len,
+                         const void *const *prefix_k, const void *const *prefix_v,
+                         const float *inv_temp, const uint64_t *seeds, void *cuda_stream);
+
+/* One denoise step of every canvas that is not done: steps 1-7 above. Canvases
+ * that are done are left unchanged. Asynchronous. dbg may be NULL. */
+dg_status dg_denoise_step(dg_ctx *ctx, const dg_schedule *sched, const dg_step_out *dbg);
+
+/* Denoise until every canvas is done (at most sched->max_steps steps each).
+ *   tokens_out  [B*C] int32, device or host memory (copied with UVA), or NULL.
+ *   steps_out   host [B] steps taken per canvas, or NULL.
+ * Synchronous. The loop runs on the device (a CUDA graph with a device-side
+ * stop flag); the host reads one flag per step batch. */
+dg_status dg_decode_block(dg_ctx *ctx, const dg_schedule *sched, int32_t *tokens_out,
+                          int32_t *steps_out);
+
+/* Copy the decode state to / from host arrays (synchronous). set_state
+ * validates token ids (< vocab) and steps (>= 0). Together with the counter-based
+ * RNG this resumes a decode bit-exactly at any step. */
+dg_status dg_canvas_get_state(dg_ctx *ctx, dg_state *host_out);
+dg_status dg_canvas_set_state(dg_ctx *ctx, const dg_state *host_in);
+
+/* Wait for the context's stream and report device-side errors (synchronous). */
+dg_status dg_canvas_sync(dg_ctx *ctx);
+
+/* Release the workspace and the context (synchronous). NULL is a no-op. */
+void dg_canvas_destroy(dg_ctx *ctx);
+
+/* Static description of a status code. */
+const char *dg_status_string(dg_status s);
+
+/* Last error message of the calling thread (empty string if none). */
+const char *dg_last_error(void);
+
+/* ABI version of the loaded library (DG_ABI_VERSION). */
+int32_t dg_abi_version(void);
+
+/* Number of GPU kernel launches queued by the most recent dg_denoise_step
+ * (for launch accounting). */
+int32_t dg_launches_per_step(const dg_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_CANVAS_H */

@@ -1,0 +1,112 @@
+"""CPU checks of the C ABI: the library loads and exports every function that
+include/*.h declares; host-side argument validation rejects bad input before
+any device work (no GPU needed for these calls)."""
+import ctypes as C
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(dg_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from token_canvas_denoising_b200 import _lib
+    if not os.path.exists(_lib.LIB_PATH):
+        from token_canvas_denoising_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("dg_canvas_init", "dg_denoise_step", "dg_decode_block", "dg_canvas_get_state",
+              "dg_canvas_set_state", "dg_canvas_destroy", "dg_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from token_canvas_denoising_b200 import _lib
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared but not exported"
+        assert n in _lib.SIGNATURES, f"{n} has no Python signature"
+
+
+def test_status_strings_and_version(lib):
+    from token_canvas_denoising_b200 import _lib
+    assert lib.dg_abi_version() == 1
+    for s in range(7):
+        assert lib.dg_status_string(s)
+    assert lib.dg_status_string(_lib.DG_ERR_OOM) == b"out of device memory"
+
+
+def _model(**kw):
+    from token_canvas_denoising_b200 import _lib
+    m = _lib.dg_model_desc()
+    m.d_model, m.n_q_heads, m.n_kv_heads, m.head_dim, m.vocab, m.dtype = 64, 2, 1, 32, 512, _lib.DG_F32
+    for k in ("embed", "wq", "wk", "wv", "wo", "lm_head"):
+        setattr(m, k, 4096)  # never dereferenced: validation fails first or no GPU
+    for k, v in kw.items():
+        setattr(m, k, v)
+    return m
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(dtype=7), 1),
+    (dict(n_q_heads=3, n_kv_heads=2), 1),
+    (dict(lm_head=None), 1),
+    (dict(embed=4097), 1),          # misaligned
+    (dict(head_dim=48), 2),         # f32 head_dim must be a multiple of 32
+    (dict(dtype=1, head_dim=64), 2),  # bf16 needs head_dim 128
+    (dict(dtype=1, head_dim=128, vocab=1000), 2),
+])
+def test_init_rejects_bad_models(lib, over, status):
+    m = _model(**over)
+    ctx = C.c_void_p()
+    plen = (C.c_int32 * 1)(0)
+    seeds = (C.c_uint64 * 1)(0)
+    st = lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None,
+                            None, C.cast(seeds, C.c_void_p), None)
+    assert st == status, lib.dg_last_error()
+    assert not ctx.value
+
+
+@pytest.mark.parametrize("batch,canvas", [(0, 16), (1, 0), (1, 257)])
+def test_init_rejects_bad_sizes(lib, batch, canvas):
+    m = _model()
+    ctx = C.c_void_p()
+    plen = (C.c_int32 * 1)(0)
+    seeds = (C.c_uint64 * 1)(0)
+    st = lib.dg_canvas_init(C.byref(ctx), C.byref(m), batch, canvas, C.cast(plen, C.c_void_p), None,
+                            None, None, C.cast(seeds, C.c_void_p), None)
+    assert st == 1
+
+
+def test_null_context_calls_fail_cleanly(lib):
+    from token_canvas_denoising_b200 import _lib
+    s = _lib.dg_schedule(48, 0.05, 1, 0)
+    assert lib.dg_denoise_step(None, C.byref(s), None) == 1
+    assert lib.dg_decode_block(None, C.byref(s), None, None) == 1
+    assert lib.dg_canvas_sync(None) == 1
+    lib.dg_canvas_destroy(None)
+
+
+def test_product_binding_has_no_fallback(monkeypatch, tmp_path):
+    """The binding raises when the library is missing instead of computing on the CPU."""
+    from token_canvas_denoising_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        _lib.load()

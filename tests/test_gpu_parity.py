@@ -1,0 +1,110 @@
+"""GPU parity of the whole denoise path against the fp64 oracle, through the C ABI.
+
+Small cases run the full decode in free-running mode (bit-exact until the
+first ambiguous decision, lock-step after it). Shapes span several tiles of
+every kernel and ragged tails (prefix lengths and canvas lengths that are not
+tile multiples).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from oracle import model as om
+from token_canvas_denoising_b200 import inputs as fx
+from tests.oracle_adapter import oracle_model, oracle_prefix, oracle_sched
+from tests.parity import run_lockstep
+
+pytestmark = pytest.mark.gpu
+
+
+def _canvas(wl):
+    from token_canvas_denoising_b200.canvas import from_workload
+    return from_workload(wl)
+
+
+def _run(cfg, adaptive=True, n_steps=None, free_running=True, check_tensors=True, wl=None):
+    from token_canvas_denoising_b200.canvas import schedule
+    wl = wl or fx.make_workload(cfg)
+    cv, keep = _canvas(wl)
+    try:
+        invT = None if cfg.inv_temp == "one" else wl.inv_temp.astype(np.float64)
+        rep, steps = run_lockstep(cfg, cv, oracle_model(wl), oracle_prefix(wl),
+                                  oracle_sched(cfg, adaptive=adaptive),
+                                  schedule(cfg.max_steps, cfg.stop_entropy, adaptive), invT,
+                                  n_steps=n_steps, free_running=free_running,
+                                  check_tensors=check_tensors)
+    finally:
+        cv.close()
+    assert not rep.errors, "\n".join(rep.errors[:20])
+    return rep, steps
+
+
+@pytest.mark.parametrize("adaptive", [True, False])
+def test_tiny_f32_full_decode(adaptive):
+    rep, steps = _run(fx.CONFIGS["tiny"], adaptive=adaptive)
+    assert 1 <= steps <= 8
+
+
+def test_f32_ragged_multi_request():
+    cfg = fx.Config("f32_ragged", B=3, C=37, S=(0, 45, 130), d=96, Hq=4, Hk=2, h=64, V=1000,
+                    dtype="f32", max_steps=6, weight_seed=9, canvas_seeds=(5, 6, 7))
+    _run(cfg)
+
+
+def test_bf16_small_multi_tile():
+    cfg = fx.Config("bf16_small", B=2, C=200, S=(300, 77), d=256, Hq=4, Hk=2, h=128, V=4096,
+                    dtype="bf16", max_steps=12, weight_seed=13, canvas_seeds=(21, 22))
+    _run(cfg, n_steps=4)
+
+
+def test_bf16_canvas256_first_steps():
+    """The canvas256 workload (B1 C256 S1024 d2048 16/8 heads, V32768): the
+    first steps in lock-step against the oracle."""
+    _run(fx.CONFIGS["canvas256"], n_steps=3, free_running=False)
+
+
+def test_decode_block_matches_stepping():
+    """dg_decode_block (device loop) ends in the same state as single steps."""
+    from token_canvas_denoising_b200.canvas import from_workload, schedule
+    cfg = fx.Config("loop", B=2, C=24, S=(10, 33), d=64, Hq=2, Hk=1, h=32, V=300, dtype="f32",
+                    max_steps=7, weight_seed=3, canvas_seeds=(1, 2))
+    wl = fx.make_workload(cfg)
+    s = schedule(cfg.max_steps, cfg.stop_entropy, True)
+    a, _ = from_workload(wl)
+    b, _ = from_workload(wl)
+    try:
+        toks, steps = a.decode(s)
+        while not np.all(b.get_state()["done"]):
+            b.step(s)
+        sb = b.get_state()
+        assert np.array_equal(toks.numpy(), sb["tokens"])
+        assert steps == sb["step"].tolist()
+        assert all(1 <= x <= cfg.max_steps for x in steps)
+    finally:
+        a.close()
+        b.close()
+
+
+def test_state_roundtrip_resumes_bit_exactly():
+    from token_canvas_denoising_b200.canvas import from_workload, schedule
+    cfg = fx.Config("resume", B=1, C=40, S=(20,), d=64, Hq=2, Hk=1, h=32, V=256, dtype="f32",
+                    max_steps=8, weight_seed=4, canvas_seeds=(11,))
+    wl = fx.make_workload(cfg)
+    s = schedule(cfg.max_steps, cfg.stop_entropy, False)
+    a, _ = from_workload(wl)
+    b, _ = from_workload(wl)
+    try:
+        for _ in range(3):
+            a.step(s)
+        mid = a.get_state()
+        b.set_state(mid)
+        for _ in range(2):
+            a.step(s)
+            b.step(s)
+        sa, sb = a.get_state(), b.get_state()
+        for k in sa:
+            assert np.array_equal(sa[k], sb[k]), k
+    finally:
+        a.close()
+        b.close()

@@ -1,0 +1,150 @@
+"""Python binding of libdgcanvas: a thin object over the C ABI.
+
+PyTorch provides device memory and streams only; the denoise path runs in the
+CUDA library (see include/dg_canvas.h for what each call computes).
+"""
+import ctypes as C
+
+import numpy as np
+import torch
+
+from . import _lib as L
+
+_DT = {"f32": L.DG_F32, "bf16": L.DG_BF16}
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
+
+
+def to_device(arr, dtype, device):
+    """numpy storage array (uint16 bf16 bits or float32) -> contiguous torch tensor."""
+    t = torch.from_numpy(np.ascontiguousarray(arr))
+    if dtype == "bf16":
+        t = t.view(torch.bfloat16)
+    return t.to(device, non_blocking=False).contiguous()
+
+
+def schedule(max_steps=48, stop_entropy=0.05, adaptive_stop=True):
+    return L.dg_schedule(int(max_steps), float(stop_entropy), 1 if adaptive_stop else 0, L.DG_SCHED_CEIL)
+
+
+class DenoiseCanvas:
+    """A decode context for B canvases of C positions.
+
+    weights: dict of device tensors in the storage dtype: embed, wq, wk, wv, wo,
+    lm_head (+ w_router, w_gate, w_up, w_down for MoE). prefix_k / prefix_v:
+    lists of B device tensors [S_b, Hk, h]. inv_temp: device f32 [B*C] or None.
+    """
+
+    def __init__(self, weights, *, d_model, n_q_heads, n_kv_heads, head_dim, vocab, dtype,
+                 canvas_len, prefix_k, prefix_v, seeds, inv_temp=None, n_experts=0, top_k=0,
+                 moe_inter=0, n_shared=0, stream=None):
+        self._lib = L.load()
+        self.B = len(seeds)
+        self.C = int(canvas_len)
+        self.M = self.B * self.C
+        self.dtype = dtype
+        self._keep = [weights, prefix_k, prefix_v, inv_temp]  # keep caller memory alive
+        m = L.dg_model_desc()
+        m.d_model, m.n_q_heads, m.n_kv_heads, m.head_dim, m.vocab = d_model, n_q_heads, n_kv_heads, head_dim, vocab
+        m.dtype = _DT[dtype]
+        for k in ("embed", "wq", "wk", "wv", "wo", "lm_head"):
+            setattr(m, k, weights[k].data_ptr())
+        m.n_experts, m.top_k, m.moe_inter, m.n_shared = n_experts, top_k, moe_inter, n_shared
+        if n_experts:
+            for k in ("w_router", "w_gate", "w_up", "w_down"):
+                setattr(m, k, weights[k].data_ptr())
+        self._model = m
+        plen = (C.c_int32 * self.B)(*[int(t.shape[0]) if t is not None else 0 for t in prefix_k])
+        pk = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_k])
+        pv = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_v])
+        sd = (C.c_uint64 * self.B)(*[int(s) for s in seeds])
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        ctx = C.c_void_p()
+        st = self._lib.dg_canvas_init(C.byref(ctx), C.byref(m), self.B, self.C, C.cast(plen, C.c_void_p),
+                                      C.cast(pk, C.c_void_p), C.cast(pv, C.c_void_p), _ptr(inv_temp),
+                                      C.cast(sd, C.c_void_p), C.c_void_p(self.stream.cuda_stream))
+        L.check(st, "dg_canvas_init")
+        self._ctx = ctx
+
+    # ------------------------------------------------------------------
+    def step(self, sched, debug=False):
+        """One denoise step; with debug=True returns the per-step outputs."""
+        out = None
+        dbg = None
+        if debug:
+            dev = torch.device("cuda", torch.cuda.current_device())
+            sdt = torch.float32 if self.dtype == "f32" else torch.bfloat16
+            out = {
+                "ent": torch.empty(self.M, dtype=torch.float32, device=dev),
+                "argmax": torch.empty(self.M, dtype=torch.int32, device=dev),
+                "freeze_mask": torch.empty(self.M, dtype=torch.uint8, device=dev),
+                "attn_out": torch.empty(self.M, self._model.n_q_heads * self._model.head_dim, dtype=sdt, device=dev),
+                "hidden": torch.empty(self.M, self._model.d_model, dtype=sdt, device=dev),
+            }
+            dbg = L.dg_step_out(*[_ptr(out[k]) for k in ("ent", "argmax", "freeze_mask", "attn_out", "hidden")])
+        st = self._lib.dg_denoise_step(self._ctx, C.byref(sched), C.byref(dbg) if dbg is not None else None)
+        L.check(st, "dg_denoise_step")
+        return out
+
+    def decode(self, sched, tokens_out=None):
+        """Denoise to completion. tokens_out: torch tensor (device or host int32
+        [B*C]) or None for a fresh host tensor. Returns (tokens, steps)."""
+        if tokens_out is None:
+            tokens_out = torch.empty(self.M, dtype=torch.int32)
+        steps = (C.c_int32 * self.B)()
+        st = self._lib.dg_decode_block(self._ctx, C.byref(sched), _ptr(tokens_out), C.cast(steps, C.c_void_p))
+        L.check(st, "dg_decode_block")
+        return tokens_out, list(steps)
+
+    def get_state(self):
+        s = {"tokens": np.zeros(self.M, np.int32), "frozen": np.zeros(self.M, np.uint8),
+             "step": np.zeros(self.B, np.int32), "seed": np.zeros(self.B, np.uint64),
+             "done": np.zeros(self.B, np.uint8)}
+        hs = L.dg_state(*[s[k].ctypes.data for k in ("tokens", "frozen", "step", "seed", "done")])
+        L.check(self._lib.dg_canvas_get_state(self._ctx, C.byref(hs)), "dg_canvas_get_state")
+        return s
+
+    def set_state(self, s):
+        arrs = {"tokens": np.ascontiguousarray(s["tokens"], np.int32).reshape(-1),
+                "frozen": np.ascontiguousarray(s["frozen"], np.uint8).reshape(-1),
+                "step": np.ascontiguousarray(s["step"], np.int32).reshape(-1),
+                "seed": np.ascontiguousarray(s["seed"], np.uint64).reshape(-1),
+                "done": np.ascontiguousarray(s["done"], np.uint8).reshape(-1)}
+        hs = L.dg_state(*[arrs[k].ctypes.data for k in ("tokens", "frozen", "step", "seed", "done")])
+        L.check(self._lib.dg_canvas_set_state(self._ctx, C.byref(hs)), "dg_canvas_set_state")
+
+    def sync(self):
+        L.check(self._lib.dg_canvas_sync(self._ctx), "dg_canvas_sync")
+
+    @property
+    def launches_per_step(self):
+        return int(self._lib.dg_launches_per_step(self._ctx))
+
+    def close(self):
+        if getattr(self, "_ctx", None):
+            self._lib.dg_canvas_destroy(self._ctx)
+            self._ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def from_workload(wl, device=None, stream=None):
+    """Upload a seeded Workload (token_canvas_denoising_b200.inputs) and create a
+    DenoiseCanvas over it. Returns (canvas, device tensors)."""
+    c = wl.cfg
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    w = {k: to_device(v, c.dtype, device) for k, v in wl.weights.items()}
+    pk = [to_device(x, c.dtype, device) for x in wl.prefix_k]
+    pv = [to_device(x, c.dtype, device) for x in wl.prefix_v]
+    invT = None if c.inv_temp == "one" else torch.from_numpy(wl.inv_temp).to(device)
+    cv = DenoiseCanvas(w, d_model=c.d, n_q_heads=c.Hq, n_kv_heads=c.Hk, head_dim=c.h, vocab=c.V,
+                       dtype=c.dtype, canvas_len=c.C, prefix_k=pk, prefix_v=pv, seeds=list(wl.seeds),
+                       inv_temp=invT, n_experts=c.n_experts, top_k=c.top_k, moe_inter=c.moe_inter,
+                       n_shared=c.n_shared, stream=stream)
+    return cv, {"weights": w, "prefix_k": pk, "prefix_v": pv, "inv_temp": invT}

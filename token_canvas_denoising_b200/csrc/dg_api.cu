@@ -1,0 +1,356 @@
+// C ABI of libdgcanvas: argument validation, workspace, the per-step launch
+// sequence, the device-side decode loop and state transfer. The operations
+// themselves are described in include/dg_canvas.h.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "dg_internal.cuh"
+
+namespace dg {
+
+static thread_local std::string g_last_error;
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
+}  // namespace dg
+
+using dg::set_last_error;
+
+#define DG_CUDA_RET(expr)                                                              \
+  do {                                                                                 \
+    cudaError_t e__ = (expr);                                                          \
+    if (e__ != cudaSuccess) {                                                          \
+      set_last_error(std::string(#expr) + ": " + cudaGetErrorString(e__));             \
+      return DG_ERR_CUDA;                                                              \
+    }                                                                                  \
+  } while (0)
+
+#define DG_ARG(cond, msg)                          \
+  do {                                             \
+    if (!(cond)) {                                 \
+      set_last_error(std::string("invalid argument: ") + (msg)); \
+      return DG_ERR_INVALID_ARG;                   \
+    }                                              \
+  } while (0)
+
+#define DG_UNSUP(cond, msg)                        \
+  do {                                             \
+    if (!(cond)) {                                 \
+      set_last_error(std::string("unsupported: ") + (msg)); \
+      return DG_ERR_UNSUPPORTED;                   \
+    }                                              \
+  } while (0)
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bump allocator over one cudaMalloc'd block; every buffer 256-byte aligned.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T> T* take(size_t count) {
+    off = (off + 255) & ~size_t(255);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+void layout_workspace(dg_ctx* c, void* base, size_t* total) {
+  Carver w(base);
+  const size_t M = c->M, d = c->m.d_model;
+  const size_t qd = (size_t)c->m.n_q_heads * c->m.head_dim, kd = (size_t)c->m.n_kv_heads * c->m.head_dim;
+  c->tok = w.take<int32_t>(M);
+  c->frozen = w.take<uint8_t>(M);
+  c->step = w.take<int32_t>(c->B);
+  c->seed = w.take<uint64_t>(c->B);
+  c->done = w.take<uint8_t>(c->B);
+  c->err = w.take<int32_t>(1);
+  c->all_done = w.take<int32_t>(1);
+  c->counters = w.take<uint32_t>(c->B + 1);
+  c->d_prefix = w.take<dg::PrefixDesc>(c->B);
+  c->X = w.take<char>(M * d * c->es);
+  c->Q = w.take<char>(M * qd * c->es);
+  c->Kc = w.take<char>(M * kd * c->es);
+  c->Vc = w.take<char>(M * kd * c->es);
+  c->O = w.take<char>(M * qd * c->es);
+  c->Hs = w.take<char>(M * d * c->es);
+  c->Hs2 = c->m.n_experts ? w.take<char>(M * d * c->es) : nullptr;
+  c->lm.rec = w.take<dg::LmRec>(M * (size_t)c->lm.P);
+  c->ent = w.take<float>(M);
+  c->am = w.take<int32_t>(M);
+  c->fmask = w.take<uint8_t>(M);
+  *total = w.off + 256;
+}
+
+dg_status validate_model(const dg_model_desc* m) {
+  DG_ARG(m != nullptr, "model is NULL");
+  DG_ARG(m->dtype == DG_F32 || m->dtype == DG_BF16, "dtype must be DG_F32 or DG_BF16");
+  DG_ARG(m->d_model > 0 && m->n_q_heads > 0 && m->n_kv_heads > 0 && m->head_dim > 0 && m->vocab > 1,
+         "dimensions must be positive (vocab >= 2)");
+  DG_ARG(m->n_q_heads % m->n_kv_heads == 0, "n_q_heads must be a multiple of n_kv_heads");
+  DG_ARG(m->embed && m->wq && m->wk && m->wv && m->wo && m->lm_head, "a weight pointer is NULL");
+  DG_ARG(aligned16(m->embed) && aligned16(m->wq) && aligned16(m->wk) && aligned16(m->wv) &&
+             aligned16(m->wo) && aligned16(m->lm_head),
+         "weight pointers must be 16-byte aligned");
+  DG_UNSUP(m->d_model % 8 == 0, "d_model must be a multiple of 8");
+  if (m->dtype == DG_F32) {
+    DG_UNSUP(m->head_dim % 32 == 0 && m->head_dim <= 128, "f32 head_dim must be 32, 64, 96 or 128");
+  } else {
+    DG_UNSUP(m->head_dim == 128, "bf16 head_dim must be 128");
+    DG_UNSUP(m->d_model % 64 == 0, "bf16 d_model must be a multiple of 64");
+    DG_UNSUP(m->vocab % 256 == 0, "bf16 vocab must be a multiple of 256");
+  }
+  if (m->n_experts != 0) {
+    DG_ARG(m->n_experts > 0 && m->top_k > 0 && m->top_k <= m->n_experts && m->moe_inter > 0 &&
+               m->n_shared >= 0,
+           "MoE sizes");
+    DG_ARG(m->w_router && m->w_gate && m->w_up && m->w_down, "an MoE weight pointer is NULL");
+    DG_UNSUP(false, "MoE FFN is not available in this build");
+  }
+  return DG_OK;
+}
+
+dg_status validate_sched(const dg_schedule* s) {
+  DG_ARG(s != nullptr, "schedule is NULL");
+  DG_ARG(s->max_steps >= 1 && s->max_steps <= 1024, "max_steps must be in [1, 1024]");
+  DG_ARG(s->kind == DG_SCHED_CEIL, "unknown schedule kind");
+  DG_ARG(s->stop_entropy == s->stop_entropy, "stop_entropy is NaN");
+  return DG_OK;
+}
+
+dg_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error(std::string(what) + ": " + cudaGetErrorString(e));
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
+}
+
+// The launch sequence of one denoise step (steps 1-7 of the header).
+dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) {
+  const int M = c->M, d = c->m.d_model;
+  const int qd = c->m.n_q_heads * c->m.head_dim, kd = c->m.n_kv_heads * c->m.head_dim;
+  c->launches = 0;
+  dg::launch_embed(c);
+  dg::launch_linear_simple(c, c->X, c->m.wq, nullptr, c->Q, M, qd, d);
+  dg::launch_linear_simple(c, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
+  dg::launch_linear_simple(c, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
+  dg::launch_attention_simple(c);
+  dg::launch_linear_simple(c, c->O, c->m.wo, c->X, c->Hs, M, d, qd);
+  const void* hs = c->Hs;
+  dg::launch_lmhead_simple(c, hs);
+  dg::launch_merge_select(c, s, dbg && dbg->freeze_mask ? dbg->freeze_mask : nullptr);
+  dg_status st = check_launch("denoise step launch");
+  if (st != DG_OK) return st;
+  if (dbg) {
+    if (dbg->ent) DG_CUDA_RET(cudaMemcpyAsync(dbg->ent, c->ent, M * sizeof(float), cudaMemcpyDeviceToDevice, c->stream));
+    if (dbg->argmax) DG_CUDA_RET(cudaMemcpyAsync(dbg->argmax, c->am, M * sizeof(int32_t), cudaMemcpyDeviceToDevice, c->stream));
+    if (dbg->attn_out) DG_CUDA_RET(cudaMemcpyAsync(dbg->attn_out, c->O, (size_t)M * qd * c->es, cudaMemcpyDeviceToDevice, c->stream));
+    if (dbg->hidden) DG_CUDA_RET(cudaMemcpyAsync(dbg->hidden, hs, (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, c->stream));
+  }
+  return DG_OK;
+}
+
+dg_status read_device_error(dg_ctx* c) {
+  int32_t e = 0;
+  DG_CUDA_RET(cudaMemcpyAsync(&e, c->err, sizeof(e), cudaMemcpyDeviceToHost, c->stream));
+  DG_CUDA_RET(cudaStreamSynchronize(c->stream));
+  if (e == 0) return DG_OK;
+  char buf[96];
+  snprintf(buf, sizeof buf, "device-side check failed (code %d)", e);
+  set_last_error(buf);
+  return e == dg::kDevWaitTimeout ? DG_ERR_TIMEOUT : DG_ERR_DEVICE_CHECK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t dg_abi_version(void) { return DG_ABI_VERSION; }
+
+const char* dg_last_error(void) { return dg::g_last_error.c_str(); }
+
+const char* dg_status_string(dg_status s) {
+  switch (s) {
+    case DG_OK: return "ok";
+    case DG_ERR_INVALID_ARG: return "invalid argument";
+    case DG_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case DG_ERR_OOM: return "out of device memory";
+    case DG_ERR_CUDA: return "CUDA error";
+    case DG_ERR_TIMEOUT: return "device wait timed out";
+    case DG_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+int32_t dg_launches_per_step(const dg_ctx* ctx) { return ctx ? ctx->launches : 0; }
+
+dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch, int32_t canvas_len,
+                         const int32_t* prefix_len, const void* const* prefix_k,
+                         const void* const* prefix_v, const float* inv_temp, const uint64_t* seeds,
+                         void* cuda_stream) {
+  DG_ARG(out != nullptr, "out is NULL");
+  *out = nullptr;
+  dg_status st = validate_model(model);
+  if (st != DG_OK) return st;
+  DG_ARG(batch >= 1 && batch <= 4096, "batch must be in [1, 4096]");
+  DG_ARG(canvas_len >= 1 && canvas_len <= 256, "canvas_len must be in [1, 256]");
+  DG_ARG(prefix_len && seeds, "prefix_len / seeds is NULL");
+  for (int b = 0; b < batch; ++b) {
+    DG_ARG(prefix_len[b] >= 0 && prefix_len[b] <= (1 << 24), "prefix_len out of range");
+    if (prefix_len[b] > 0) {
+      DG_ARG(prefix_k && prefix_v && prefix_k[b] && prefix_v[b], "prefix K/V pointer is NULL");
+      DG_ARG(aligned16(prefix_k[b]) && aligned16(prefix_v[b]), "prefix K/V must be 16-byte aligned");
+    }
+  }
+  if (inv_temp) DG_ARG(aligned16(inv_temp), "inv_temp must be 16-byte aligned");
+
+  dg_ctx* c = new dg_ctx();
+  c->m = *model;
+  c->B = batch;
+  c->C = canvas_len;
+  c->M = batch * canvas_len;
+  c->es = model->dtype == DG_F32 ? 4 : 2;
+  c->inv_temp = inv_temp;
+  c->stream = static_cast<cudaStream_t>(cuda_stream);
+  for (int b = 0; b < batch; ++b) {
+    c->S.push_back(prefix_len[b]);
+    c->pk.push_back(prefix_len[b] ? prefix_k[b] : nullptr);
+    c->pv.push_back(prefix_len[b] ? prefix_v[b] : nullptr);
+    c->max_S = std::max(c->max_S, (int)prefix_len[b]);
+  }
+  auto fail = [&](dg_status s) { dg_canvas_destroy(c); return s; };
+  if (cudaGetDevice(&c->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+    set_last_error("no usable CUDA device");
+    return fail(DG_ERR_CUDA);
+  }
+  c->lm.P = std::max(1, std::min(128, model->vocab / 1024));
+
+  size_t total = 0;
+  layout_workspace(c, nullptr, &total);
+  const char* lim = std::getenv("DG_WORKSPACE_LIMIT_MB");
+  if (lim && (double)total > std::atof(lim) * 1048576.0) {
+    set_last_error("workspace exceeds DG_WORKSPACE_LIMIT_MB");
+    return fail(DG_ERR_OOM);
+  }
+  if (cudaMalloc(&c->ws, total) != cudaSuccess) {
+    cudaGetLastError();
+    set_last_error("cudaMalloc of the workspace failed");
+    return fail(DG_ERR_OOM);
+  }
+  c->ws_bytes = total;
+  layout_workspace(c, c->ws, &total);
+
+  std::vector<dg::PrefixDesc> pd(batch);
+  for (int b = 0; b < batch; ++b) pd[b] = {c->pk[b], c->pv[b], c->S[b], 0};
+  std::vector<uint32_t> zeros(batch + 1, 0);
+  if (cudaMemcpyAsync(c->d_prefix, pd.data(), batch * sizeof(dg::PrefixDesc), cudaMemcpyHostToDevice, c->stream) != cudaSuccess ||
+      cudaMemcpyAsync(c->seed, seeds, batch * sizeof(uint64_t), cudaMemcpyHostToDevice, c->stream) != cudaSuccess ||
+      cudaMemsetAsync(c->counters, 0, (batch + 1) * sizeof(uint32_t), c->stream) != cudaSuccess ||
+      cudaMemsetAsync(c->err, 0, sizeof(int32_t), c->stream) != cudaSuccess) {
+    set_last_error("initial copies failed");
+    return fail(DG_ERR_CUDA);
+  }
+  dg::launch_init_canvas(c);
+  st = check_launch("init canvas");
+  if (st != DG_OK) return fail(st);
+  if (cudaStreamSynchronize(c->stream) != cudaSuccess) {
+    set_last_error("init synchronize failed");
+    return fail(DG_ERR_CUDA);
+  }
+  *out = c;
+  return DG_OK;
+}
+
+dg_status dg_denoise_step(dg_ctx* ctx, const dg_schedule* sched, const dg_step_out* dbg) {
+  DG_ARG(ctx != nullptr, "ctx is NULL");
+  dg_status st = validate_sched(sched);
+  if (st != DG_OK) return st;
+  return enqueue_step(ctx, *sched, dbg);
+}
+
+dg_status dg_decode_block(dg_ctx* ctx, const dg_schedule* sched, int32_t* tokens_out, int32_t* steps_out) {
+  DG_ARG(ctx != nullptr, "ctx is NULL");
+  dg_status st = validate_sched(sched);
+  if (st != DG_OK) return st;
+  // Every canvas stops within max_steps (the freeze count reaches all
+  // remaining positions at the last step), so max_steps launches suffice; the
+  // device flag lets the host stop early without a per-step round trip.
+  int32_t all = 0;
+  DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  int launched = 0;
+  while (!all && launched < sched->max_steps) {
+    const int batch = std::min(4, sched->max_steps - launched);
+    for (int i = 0; i < batch; ++i) {
+      st = enqueue_step(ctx, *sched, nullptr);
+      if (st != DG_OK) return st;
+    }
+    launched += batch;
+    DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->stream));
+    DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  }
+  st = read_device_error(ctx);
+  if (st != DG_OK) return st;
+  if (tokens_out)
+    DG_CUDA_RET(cudaMemcpyAsync(tokens_out, ctx->tok, ctx->M * sizeof(int32_t), cudaMemcpyDefault, ctx->stream));
+  if (steps_out)
+    DG_CUDA_RET(cudaMemcpyAsync(steps_out, ctx->step, ctx->B * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  return DG_OK;
+}
+
+dg_status dg_canvas_get_state(dg_ctx* ctx, dg_state* h) {
+  DG_ARG(ctx && h, "NULL argument");
+  DG_ARG(h->tokens && h->frozen && h->step && h->seed && h->done, "a state array is NULL");
+  DG_CUDA_RET(cudaMemcpyAsync(h->tokens, ctx->tok, ctx->M * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->frozen, ctx->frozen, ctx->M, cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->step, ctx->step, ctx->B * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->seed, ctx->seed, ctx->B * sizeof(uint64_t), cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->done, ctx->done, ctx->B, cudaMemcpyDeviceToHost, ctx->stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  return read_device_error(ctx);
+}
+
+dg_status dg_canvas_set_state(dg_ctx* ctx, const dg_state* h) {
+  DG_ARG(ctx && h, "NULL argument");
+  DG_ARG(h->tokens && h->frozen && h->step && h->seed && h->done, "a state array is NULL");
+  int all = 1;
+  for (int i = 0; i < ctx->M; ++i) DG_ARG(h->tokens[i] >= 0 && h->tokens[i] < ctx->m.vocab, "token id out of range");
+  for (int b = 0; b < ctx->B; ++b) {
+    DG_ARG(h->step[b] >= 0, "negative step");
+    all &= h->done[b] ? 1 : 0;
+  }
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->tok, h->tokens, ctx->M * sizeof(int32_t), cudaMemcpyHostToDevice, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->frozen, h->frozen, ctx->M, cudaMemcpyHostToDevice, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->step, h->step, ctx->B * sizeof(int32_t), cudaMemcpyHostToDevice, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->seed, h->seed, ctx->B * sizeof(uint64_t), cudaMemcpyHostToDevice, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->done, h->done, ctx->B, cudaMemcpyHostToDevice, ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->all_done, &all, sizeof(int32_t), cudaMemcpyHostToDevice, ctx->stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  return DG_OK;
+}
+
+dg_status dg_canvas_sync(dg_ctx* ctx) {
+  DG_ARG(ctx != nullptr, "ctx is NULL");
+  return read_device_error(ctx);
+}
+
+void dg_canvas_destroy(dg_ctx* ctx) {
+  if (!ctx) return;
+  if (ctx->ws) {
+    cudaStreamSynchronize(ctx->stream);
+    cudaFree(ctx->ws);
+  }
+  if (ctx->graph_exec) cudaGraphExecDestroy(ctx->graph_exec);
+  delete ctx;
+}
+
+}  // extern "C"

@@ -1,0 +1,200 @@
+// Canvas bookkeeping kernels: the initial random canvas, and the fused
+// "merge LM-head partials -> entropy/argmax -> freeze -> stop test ->
+// re-noise" tail of every denoise step.
+//
+// Method ("DiffusionGemma解析：扩散模型如何让LLM快5倍", 整片并行去噪 and
+// 自适应停步机制; "谷歌DiffusionGemma：并行生成与自纠的新突破", 工作原理):
+// positions are ordered by entropy, the most certain ones are locked to the
+// model's most likely token, every other position is re-randomised, and the
+// block stops once enough positions are settled (at most 48 steps).
+#include "dg_internal.cuh"
+
+namespace dg {
+
+// ------------------------------------------------------------------ init
+// tok[b][p] = draw(seed_b, step 0, p, b); nothing frozen; step 0; not done.
+__global__ void init_canvas_kernel(int32_t* tok, uint8_t* frozen, int32_t* step, const uint64_t* seed,
+                                   uint8_t* done, int32_t* all_done, int C, int V) {
+  const int b = blockIdx.x;
+  for (int p = threadIdx.x; p < C; p += blockDim.x) {
+    tok[b * C + p] = canvas_draw(seed[b], 0u, (uint32_t)p, (uint32_t)b, (uint32_t)V);
+    frozen[b * C + p] = 0;
+  }
+  if (threadIdx.x == 0) {
+    step[b] = 0;
+    done[b] = 0;
+    if (b == 0) *all_done = 0;
+  }
+}
+
+void launch_init_canvas(dg_ctx* c) {
+  init_canvas_kernel<<<c->B, 256, 0, c->stream>>>(c->tok, c->frozen, c->step, c->seed, c->done,
+                                                 c->all_done, c->C, c->m.vocab);
+}
+
+// ------------------------------------------------------------------ merge + select
+struct SelectArgs {
+  LmPartials part;
+  float* ent;           // [M]
+  int32_t* am;          // [M]
+  uint8_t* fmask;       // [M] or null
+  int32_t* tok;
+  uint8_t* frozen;
+  int32_t* step;
+  const uint64_t* seed;
+  uint8_t* done;
+  int32_t* all_done;
+  uint32_t* counters;   // [B + 1], zero on entry, left zero
+  int32_t* err;
+  int B, C, V, max_steps, adaptive;
+  float stop_entropy;
+};
+
+__device__ __forceinline__ EntStats load_rec(const LmRec* r) {
+  const float4 a = __ldcg(reinterpret_cast<const float4*>(r));
+  const int4 b = __ldcg(reinterpret_cast<const int4*>(r) + 1);
+  return {a.x, a.y, a.z, a.w, b.x};
+}
+
+// Grid (ceil(C/8), B), 256 threads. Phase 1: one warp per canvas row folds the
+// row's P partials (lane j takes partials j, j+32, ...; then a fixed xor
+// butterfly), giving ent = ln Z - S/Z and the argmax. Phase 2 runs in the last
+// block of each canvas to arrive: rank-by-count selection of the k smallest
+// (entropy, position) keys among unfrozen positions, freeze, stop test,
+// re-noise. The last canvas to finish sets the all-done flag.
+__global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p_row = blockIdx.x * 8 + warp;
+  if (p_row < a.C) {
+    const int r = b * a.C + p_row;
+    const LmRec* rec = a.part.rec + (size_t)r * a.part.P;
+    EntStats st = ent_empty();
+    for (int j = lane; j < a.part.P; j += 32) st = ent_merge(st, load_rec(rec + j));
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      EntStats ot;
+      ot.m = __shfl_xor_sync(0xffffffffu, st.m, o);
+      ot.z = __shfl_xor_sync(0xffffffffu, st.z, o);
+      ot.s = __shfl_xor_sync(0xffffffffu, st.s, o);
+      ot.best = __shfl_xor_sync(0xffffffffu, st.best, o);
+      ot.idx = __shfl_xor_sync(0xffffffffu, st.idx, o);
+      st = (lane & o) ? ent_merge(ot, st) : ent_merge(st, ot);
+    }
+    if (lane == 0) {
+      float e = logf(st.z) - st.s / st.z;
+      if (!isfinite(e)) set_error(a.err, kDevNanEntropy);
+      a.ent[r] = e;
+      a.am[r] = st.idx;
+    }
+  }
+  // ---- arrival: the last block of canvas b runs the selection
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(&a.counters[b], 1u);
+    s_last = (prev == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  __shared__ float s_ent[256];
+  __shared__ uint8_t s_unf[256];
+  __shared__ float s_min[8];
+  const int p = threadIdx.x;
+  const bool valid = p < a.C;
+  const int r = b * a.C + p;
+  const bool canvas_done = __ldcg(&a.done[b]) != 0;
+  if (canvas_done) {
+    if (valid && a.fmask) a.fmask[r] = 0;
+  } else {
+    float e = valid ? __ldcg(&a.ent[r]) : INFINITY;
+    if (!(e == e)) e = INFINITY;  // NaN (already flagged) orders last
+    const bool unf = valid && a.frozen[r] == 0;
+    s_ent[p] = e;
+    s_unf[p] = unf ? 1 : 0;
+    const int U = __syncthreads_count(unf);
+    const int t = a.step[b];
+    const int left = a.max_steps - t;
+    const int k = (left <= 1) ? U : (U + left - 1) / left;
+    bool F = false;
+    if (unf) {
+      int rank = 0;
+      for (int q = 0; q < a.C; ++q) {
+        const float eq = s_ent[q];
+        rank += (s_unf[q] && (eq < e || (eq == e && q < p))) ? 1 : 0;
+      }
+      F = rank < k;
+    }
+    const int amv = valid ? __ldcg(&a.am[r]) : 0;
+    if (F) {
+      a.tok[r] = amv;
+      a.frozen[r] = 1;
+    }
+    const bool rest = unf && !F;
+    // smallest entropy among positions still unfrozen after this freeze
+    float mr = rest ? e : INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mr = fminf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+    if (lane == 0) s_min[warp] = mr;
+    const int R = __syncthreads_count(rest);
+    float min_rest = s_min[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) min_rest = fminf(min_rest, s_min[w]);
+    const bool stop = (R == 0) || (a.adaptive && min_rest < a.stop_entropy);
+    if (stop) {
+      if (rest) a.tok[r] = amv;
+      if (valid) a.frozen[r] = 1;
+    } else if (rest) {
+      a.tok[r] = canvas_draw(a.seed[b], (uint32_t)(t + 1), (uint32_t)p, (uint32_t)b, (uint32_t)a.V);
+    }
+    if (valid && a.fmask) a.fmask[r] = F ? 1 : 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      a.step[b] = t + 1;
+      if (stop) a.done[b] = 1;
+    }
+  }
+  // ---- canvas finished: reset its counter; the last canvas sets all_done
+  if (threadIdx.x == 0) {
+    a.counters[b] = 0;
+    __threadfence();
+    const unsigned prev = atomicAdd(&a.counters[a.B], 1u);
+    if (prev == (unsigned)a.B - 1) {
+      __threadfence();
+      int all = 1;
+      for (int i = 0; i < a.B; ++i) all &= (__ldcg(&a.done[i]) != 0) ? 1 : 0;
+      *a.all_done = all;
+      a.counters[a.B] = 0;
+    }
+  }
+}
+
+void launch_merge_select(dg_ctx* c, const dg_schedule& s, uint8_t* fmask_out) {
+  SelectArgs a;
+  a.part = c->lm;
+  a.ent = c->ent;
+  a.am = c->am;
+  a.fmask = fmask_out;
+  a.tok = c->tok;
+  a.frozen = c->frozen;
+  a.step = c->step;
+  a.seed = c->seed;
+  a.done = c->done;
+  a.all_done = c->all_done;
+  a.counters = c->counters;
+  a.err = c->err;
+  a.B = c->B;
+  a.C = c->C;
+  a.V = c->m.vocab;
+  a.max_steps = s.max_steps;
+  a.adaptive = s.adaptive_stop;
+  a.stop_entropy = s.stop_entropy;
+  dim3 grid(ceil_div(c->C, 8), c->B);
+  merge_select_kernel<<<grid, 256, 0, c->stream>>>(a);
+  c->launches++;
+}
+
+}  // namespace dg

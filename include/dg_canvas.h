@@ -138,8 +138,14 @@ dg_status dg_canvas_init(dg_ctx **out, const dg_model_desc *model, int32_t batch
                          const float *inv_temp, const uint64_t *seeds, void *cuda_stream);
 
 /* One denoise step of every canvas that is not done: steps 1-7 above. Canvases
- * that are done are left unchanged. Asynchronous. dbg may be NULL. */
+ * that are done are left unchanged. Asynchronous. dbg may be NULL; without it
+ * the step runs as one CUDA graph launch (captured on the first call with a
+ * given schedule, so that first call must not happen inside a stream capture). */
 dg_status dg_denoise_step(dg_ctx *ctx, const dg_schedule *sched, const dg_step_out *dbg);
+
+/* Start a new block: redraw every canvas at step 0 from `seeds` (host [B]; NULL
+ * keeps the current seeds), clear the frozen and done flags. Asynchronous. */
+dg_status dg_canvas_reset(dg_ctx *ctx, const uint64_t *seeds);
 
 /* Denoise until every canvas is done (at most sched->max_steps steps each).
  *   tokens_out  [B*C] int32, device or host memory (copied with UVA), or NULL.
@@ -154,6 +160,13 @@ dg_status dg_decode_block(dg_ctx *ctx, const dg_schedule *sched, int32_t *tokens
  * RNG this resumes a decode bit-exactly at any step. */
 dg_status dg_canvas_get_state(dg_ctx *ctx, dg_state *host_out);
 dg_status dg_canvas_set_state(dg_ctx *ctx, const dg_state *host_in);
+
+/* Timing support: with n > 0 pairs of CUDA events (cudaEvent_t, created by the
+ * caller with timing enabled), step number i (counted from this call) of
+ * dg_denoise_step without debug outputs records starts[i % n] just before and
+ * stops[i % n] just after the LM-head kernel. n = 0 turns it off.
+ * Synchronous (drops the captured step graphs). */
+dg_status dg_canvas_set_timing_events(dg_ctx *ctx, int32_t n, void *const *starts, void *const *stops);
 
 /* Wait for the context's stream and report device-side errors (synchronous). */
 dg_status dg_canvas_sync(dg_ctx *ctx);

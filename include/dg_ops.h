@@ -1,0 +1,56 @@
+/*
+ * dg_ops.h -- single operations of the canvas denoise step on caller buffers,
+ * for kernel-level testing and for callers that compose their own step. Each
+ * runs the same kernels dg_denoise_step uses. Page references as in
+ * dg_canvas.h ([P1] "DiffusionGemma解析：扩散模型如何让LLM快5倍", [P3]
+ * "DiffusionGemma深度拆解：从逐字蹦到整块喷，LLM生成范式的结构性跃迁").
+ *
+ * All pointers are device memory unless marked host; all matrices row-major;
+ * dtype is DG_F32 or DG_BF16 (the storage type of every non-f32 buffer).
+ * Each call queues work on `stream` (cudaStream_t, NULL = default), allocates
+ * and frees its own temporary buffers (stream-ordered), and returns DG_OK or
+ * an error status (see dg_canvas.h); dg_last_error() has the detail. The
+ * calls do not synchronize.
+ */
+#ifndef DG_OPS_H
+#define DG_OPS_H
+
+#include <stdint.h>
+
+#include "dg_canvas.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* LM head fused with the per-row softmax entropy and argmax ([P1] 整片并行去噪):
+ *   x[r][v] = hs[r] . lm_head[v]          (f32 accumulate)
+ *   ent[r]  = H(softmax(x[r] * inv_temp[r])) in nats
+ *   argmax[r] = argmax_v x[r][v] (lowest v on ties)
+ * hs [M][d], lm_head [V][d] (dtype); inv_temp [M] f32 or NULL (= 1);
+ * ent [M] f32, argmax [M] int32 (outputs). The logits are never stored.
+ * bf16 needs d % 64 == 0 and V % 256 == 0; f32 any d % 8 == 0. */
+dg_status dg_lmhead_entropy(int32_t dtype, const void *hs, const void *lm_head, const float *inv_temp,
+                            int32_t M, int32_t d, int32_t V, float *ent, int32_t *argmax, void *stream);
+
+/* Bidirectional GQA attention of B*C canvas queries over each request's
+ * cached prompt K/V followed by the canvas K/V, no mask, scale 1/sqrt(h),
+ * query head q reading KV head q / (Hq/Hk) ([P1] 整片并行去噪 last paragraph;
+ * [P3] 架构解剖 2 and diagram).
+ *   q [B*C][Hq*h]; kc, vc [B*C][Hk*h]; prefix_len host [B];
+ *   prefix_k / prefix_v host arrays of B device pointers, each [S_b][Hk][h];
+ *   o [B*C][Hq*h] (output, dtype). bf16 needs h == 128. */
+dg_status dg_attention(int32_t dtype, const void *q, const void *kc, const void *vc, int32_t B, int32_t C,
+                       int32_t Hq, int32_t Hk, int32_t h, const int32_t *prefix_len,
+                       const void *const *prefix_k, const void *const *prefix_v, void *o, void *stream);
+
+/* out[M][N] = a[M][K] . w[N][K]^T (+ residual[M][N] if not NULL), f32
+ * accumulate, one rounding to dtype ([P3] 架构解剖 2: the canvas's K/V are
+ * re-projected every step). bf16 needs K % 64 == 0 and N % 16 == 0. */
+dg_status dg_linear(int32_t dtype, const void *a, const void *w, const void *residual, void *out,
+                    int32_t M, int32_t N, int32_t K, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_OPS_H */

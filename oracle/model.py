@@ -56,6 +56,15 @@ def dims(model):
     return (model["d"], model["Hq"], model["Hk"], model["h"], model["V"])
 
 
+def prewiden(model, keys=("wq", "wk", "wv", "wo", "lm_head")):
+    """A copy of the model dict whose `keys` hold fp64 values instead of stored
+    bits (same numbers; saves re-widening them on every call)."""
+    m = dict(model)
+    for k in keys:
+        m[k] = widen(model[k], model["dtype"])
+    return m
+
+
 def kv_head_of(q, Hq, Hk):
     """Consecutive query heads share one KV head."""
     return q // (Hq // Hk)

@@ -47,7 +47,10 @@ def round_storage(x, dtype):
 
 
 def widen(w, dtype):
-    """Stored weights (uint16 bf16 bits or float32) -> float64."""
+    """Stored weights (uint16 bf16 bits or float32) -> float64. An array that is
+    already float64 holds widened values and is returned unchanged."""
+    if getattr(w, "dtype", None) == np.float64:
+        return w
     if dtype == "bf16":
         return bf16_bits_to_f64(w)
     return np.asarray(w, dtype=np.float64)

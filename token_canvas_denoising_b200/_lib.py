@@ -51,11 +51,21 @@ SIGNATURES = {
     "dg_canvas_get_state": (C.c_int, [C.c_void_p, C.POINTER(dg_state)]),
     "dg_canvas_set_state": (C.c_int, [C.c_void_p, C.POINTER(dg_state)]),
     "dg_canvas_sync": (C.c_int, [C.c_void_p]),
+    "dg_canvas_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "dg_canvas_set_timing_events": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]),
     "dg_canvas_destroy": (None, [C.c_void_p]),
     "dg_status_string": (C.c_char_p, [C.c_int]),
     "dg_last_error": (C.c_char_p, []),
     "dg_abi_version": (C.c_int32, []),
     "dg_launches_per_step": (C.c_int32, [C.c_void_p]),
+    # include/dg_ops.h
+    "dg_lmhead_entropy": (C.c_int, [C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
+                                    C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_attention": (C.c_int, [C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
+                               C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
+                               C.c_void_p, C.c_void_p]),
+    "dg_linear": (C.c_int, [C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
+                            C.c_int32, C.c_int32, C.c_void_p]),
 }
 
 _lib = None

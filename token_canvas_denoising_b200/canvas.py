@@ -115,6 +115,23 @@ class DenoiseCanvas:
         hs = L.dg_state(*[arrs[k].ctypes.data for k in ("tokens", "frozen", "step", "seed", "done")])
         L.check(self._lib.dg_canvas_set_state(self._ctx, C.byref(hs)), "dg_canvas_set_state")
 
+    def reset(self, seeds=None):
+        """Redraw every canvas at step 0 (device side, asynchronous)."""
+        arr = None
+        if seeds is not None:
+            arr = (C.c_uint64 * self.B)(*[int(x) for x in seeds])
+        st = self._lib.dg_canvas_reset(self._ctx, C.cast(arr, C.c_void_p) if arr is not None else None)
+        L.check(st, "dg_canvas_reset")
+
+    def set_timing_events(self, starts, stops):
+        """Record torch.cuda.Event pairs around the LM-head kernel of graph steps
+        (pair i on step i mod n). Pass empty lists to turn off."""
+        n = len(starts)
+        a = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in starts])
+        b = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in stops])
+        st = self._lib.dg_canvas_set_timing_events(self._ctx, n, C.cast(a, C.c_void_p), C.cast(b, C.c_void_p))
+        L.check(st, "dg_canvas_set_timing_events")
+
     def sync(self):
         L.check(self._lib.dg_canvas_sync(self._ctx), "dg_canvas_sync")
 

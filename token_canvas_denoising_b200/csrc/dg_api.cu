@@ -63,14 +63,14 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   Carver w(base);
   const size_t M = c->M, d = c->m.d_model;
   const size_t qd = (size_t)c->m.n_q_heads * c->m.head_dim, kd = (size_t)c->m.n_kv_heads * c->m.head_dim;
-  c->tok = w.take<int32_t>(M);
-  c->frozen = w.take<uint8_t>(M);
-  c->step = w.take<int32_t>(c->B);
-  c->seed = w.take<uint64_t>(c->B);
-  c->done = w.take<uint8_t>(c->B);
+  c->cs.tok = w.take<int32_t>(M);
+  c->cs.frozen = w.take<uint8_t>(M);
+  c->cs.step = w.take<int32_t>(c->B);
+  c->cs.seed = w.take<uint64_t>(c->B);
+  c->cs.done = w.take<uint8_t>(c->B);
+  c->cs.all_done = w.take<int32_t>(1);
+  c->cs.counters = w.take<uint32_t>(c->B + 1);
   c->err = w.take<int32_t>(1);
-  c->all_done = w.take<int32_t>(1);
-  c->counters = w.take<uint32_t>(c->B + 1);
   c->d_prefix = w.take<dg::PrefixDesc>(c->B);
   c->X = w.take<char>(M * d * c->es);
   c->Q = w.take<char>(M * qd * c->es);
@@ -82,7 +82,6 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   c->lm.rec = w.take<dg::LmRec>(M * (size_t)c->lm.P);
   c->ent = w.take<float>(M);
   c->am = w.take<int32_t>(M);
-  c->fmask = w.take<uint8_t>(M);
   *total = w.off + 256;
 }
 
@@ -133,33 +132,98 @@ dg_status check_launch(const char* what) {
 
 // The launch sequence of one denoise step (steps 1-7 of the header).
 dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) {
-  const int M = c->M, d = c->m.d_model;
+  const int M = c->M, d = c->m.d_model, V = c->m.vocab;
   const int qd = c->m.n_q_heads * c->m.head_dim, kd = c->m.n_kv_heads * c->m.head_dim;
-  c->launches = 0;
-  dg::launch_embed(c);
-  dg::launch_linear_simple(c, c->X, c->m.wq, nullptr, c->Q, M, qd, d);
-  dg::launch_linear_simple(c, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
-  dg::launch_linear_simple(c, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
-  dg::launch_attention_simple(c);
-  dg::launch_linear_simple(c, c->O, c->m.wo, c->X, c->Hs, M, d, qd);
+  const int dt = c->m.dtype;
+  dg::Exec& ex = c->ex;
+  ex.launches = 0;
+  dg::launch_embed(ex, dt, c->m.embed, c->cs.tok, c->X, M, d, V);
+  dg::launch_linear_simple(ex, dt, c->X, c->m.wq, nullptr, c->Q, M, qd, d);
+  dg::launch_linear_simple(ex, dt, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
+  dg::launch_linear_simple(ex, dt, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
+  dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
+  dg::launch_attention_simple(ex, dt, c->Q, c->d_prefix, c->Kc, c->Vc, c->O, sh);
+  dg::launch_linear_simple(ex, dt, c->O, c->m.wo, c->X, c->Hs, M, d, qd);
   const void* hs = c->Hs;
-  dg::launch_lmhead_simple(c, hs);
-  dg::launch_merge_select(c, s, dbg && dbg->freeze_mask ? dbg->freeze_mask : nullptr);
+  // inside a stream capture, only an "external" record becomes an event node
+  if (c->cur_ev_start) DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start, ex.stream, cudaEventRecordExternal));
+  if (dt == DG_BF16)
+    dg::launch_lmhead_tc(ex, c->tm_lm_a, c->tm_lm_b, c->lm, c->inv_temp, M, d, V);
+  else
+    dg::launch_lmhead_simple(ex, dt, hs, c->m.lm_head, c->inv_temp, c->lm, M, d, V);
+  if (c->cur_ev_stop) DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_stop, ex.stream, cudaEventRecordExternal));
+  dg::launch_merge_select(ex, c->lm, c->ent, c->am, dbg ? dbg->freeze_mask : nullptr, &c->cs, &s, c->B, c->C, V);
+  c->launches = ex.launches;
   dg_status st = check_launch("denoise step launch");
   if (st != DG_OK) return st;
   if (dbg) {
-    if (dbg->ent) DG_CUDA_RET(cudaMemcpyAsync(dbg->ent, c->ent, M * sizeof(float), cudaMemcpyDeviceToDevice, c->stream));
-    if (dbg->argmax) DG_CUDA_RET(cudaMemcpyAsync(dbg->argmax, c->am, M * sizeof(int32_t), cudaMemcpyDeviceToDevice, c->stream));
-    if (dbg->attn_out) DG_CUDA_RET(cudaMemcpyAsync(dbg->attn_out, c->O, (size_t)M * qd * c->es, cudaMemcpyDeviceToDevice, c->stream));
-    if (dbg->hidden) DG_CUDA_RET(cudaMemcpyAsync(dbg->hidden, hs, (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, c->stream));
+    if (dbg->ent) DG_CUDA_RET(cudaMemcpyAsync(dbg->ent, c->ent, M * sizeof(float), cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->argmax) DG_CUDA_RET(cudaMemcpyAsync(dbg->argmax, c->am, M * sizeof(int32_t), cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->attn_out) DG_CUDA_RET(cudaMemcpyAsync(dbg->attn_out, c->O, (size_t)M * qd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->hidden) DG_CUDA_RET(cudaMemcpyAsync(dbg->hidden, hs, (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, ex.stream));
   }
+  return DG_OK;
+}
+
+bool same_sched(const dg_schedule& a, const dg_schedule& b) {
+  return a.max_steps == b.max_steps && a.stop_entropy == b.stop_entropy && a.adaptive_stop == b.adaptive_stop &&
+         a.kind == b.kind;
+}
+
+void drop_graphs(dg_ctx* c) {
+  for (auto g : c->graphs)
+    if (g) cudaGraphExecDestroy(g);
+  c->graphs.clear();
+}
+
+// One step without debug outputs: a CUDA graph of the whole launch sequence,
+// captured on a private stream the first time (and again when the schedule
+// changes), then launched on the caller's stream. With timing events set,
+// graph variant i records event pair i around the LM-head kernel, and step n
+// uses variant n mod (number of pairs).
+dg_status launch_step_graph(dg_ctx* c, const dg_schedule& s) {
+  const size_t nvar = std::max<size_t>(1, c->ev_start.size());
+  if (c->graphs.size() != nvar || !same_sched(c->graph_sched, s)) {
+    drop_graphs(c);
+    c->graphs.assign(nvar, nullptr);
+    c->graph_sched = s;
+  }
+  const size_t v = (size_t)(c->step_launch_count % (long long)nvar);
+  if (!c->graphs[v]) {
+    if (!c->capture_stream) DG_CUDA_RET(cudaStreamCreateWithFlags(&c->capture_stream, cudaStreamNonBlocking));
+    cudaStream_t user = c->ex.stream;
+    c->ex.stream = c->capture_stream;
+    c->cur_ev_start = c->ev_start.empty() ? nullptr : c->ev_start[v];
+    c->cur_ev_stop = c->ev_stop.empty() ? nullptr : c->ev_stop[v];
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(c->capture_stream, cudaStreamCaptureModeThreadLocal);
+    dg_status st = DG_OK;
+    if (e == cudaSuccess) {
+      st = enqueue_step(c, s, nullptr);
+      e = cudaStreamEndCapture(c->capture_stream, &g);
+    }
+    c->ex.stream = user;
+    c->cur_ev_start = c->cur_ev_stop = nullptr;
+    if (st != DG_OK) {
+      if (g) cudaGraphDestroy(g);
+      return st;
+    }
+    DG_CUDA_RET(e);
+    e = cudaGraphInstantiate(&c->graphs[v], g, 0);
+    cudaGraphDestroy(g);
+    DG_CUDA_RET(e);
+    c->graph_launches = c->launches;
+  }
+  DG_CUDA_RET(cudaGraphLaunch(c->graphs[v], c->ex.stream));
+  c->step_launch_count++;
+  c->launches = c->graph_launches;
   return DG_OK;
 }
 
 dg_status read_device_error(dg_ctx* c) {
   int32_t e = 0;
-  DG_CUDA_RET(cudaMemcpyAsync(&e, c->err, sizeof(e), cudaMemcpyDeviceToHost, c->stream));
-  DG_CUDA_RET(cudaStreamSynchronize(c->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(&e, c->err, sizeof(e), cudaMemcpyDeviceToHost, c->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(c->ex.stream));
   if (e == 0) return DG_OK;
   char buf[96];
   snprintf(buf, sizeof buf, "device-side check failed (code %d)", e);
@@ -217,7 +281,7 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   c->M = batch * canvas_len;
   c->es = model->dtype == DG_F32 ? 4 : 2;
   c->inv_temp = inv_temp;
-  c->stream = static_cast<cudaStream_t>(cuda_stream);
+  c->ex.stream = static_cast<cudaStream_t>(cuda_stream);
   for (int b = 0; b < batch; ++b) {
     c->S.push_back(prefix_len[b]);
     c->pk.push_back(prefix_len[b] ? prefix_k[b] : nullptr);
@@ -226,11 +290,15 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   }
   auto fail = [&](dg_status s) { dg_canvas_destroy(c); return s; };
   if (cudaGetDevice(&c->device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+      cudaDeviceGetAttribute(&c->ex.sm_count, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+    cudaGetLastError();
     set_last_error("no usable CUDA device");
     return fail(DG_ERR_CUDA);
   }
-  c->lm.P = std::max(1, std::min(128, model->vocab / 1024));
+  if (model->dtype == DG_BF16)
+    c->lm.P = dg::lmhead_tc_partitions(c->M, model->vocab, c->ex.sm_count);
+  else
+    c->lm.P = std::max(1, std::min(128, model->vocab / 1024));
 
   size_t total = 0;
   layout_workspace(c, nullptr, &total);
@@ -246,21 +314,26 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   }
   c->ws_bytes = total;
   layout_workspace(c, c->ws, &total);
+  c->ex.err = c->err;
+  if (model->dtype == DG_BF16 &&
+      !dg::lmhead_tc_prepare(c->Hs, model->lm_head, c->M, model->d_model, model->vocab, &c->tm_lm_a, &c->tm_lm_b))
+    return fail(DG_ERR_CUDA);
 
   std::vector<dg::PrefixDesc> pd(batch);
   for (int b = 0; b < batch; ++b) pd[b] = {c->pk[b], c->pv[b], c->S[b], 0};
   std::vector<uint32_t> zeros(batch + 1, 0);
-  if (cudaMemcpyAsync(c->d_prefix, pd.data(), batch * sizeof(dg::PrefixDesc), cudaMemcpyHostToDevice, c->stream) != cudaSuccess ||
-      cudaMemcpyAsync(c->seed, seeds, batch * sizeof(uint64_t), cudaMemcpyHostToDevice, c->stream) != cudaSuccess ||
-      cudaMemsetAsync(c->counters, 0, (batch + 1) * sizeof(uint32_t), c->stream) != cudaSuccess ||
-      cudaMemsetAsync(c->err, 0, sizeof(int32_t), c->stream) != cudaSuccess) {
+  cudaStream_t sm = c->ex.stream;
+  if (cudaMemcpyAsync(c->d_prefix, pd.data(), batch * sizeof(dg::PrefixDesc), cudaMemcpyHostToDevice, sm) != cudaSuccess ||
+      cudaMemcpyAsync(c->cs.seed, seeds, batch * sizeof(uint64_t), cudaMemcpyHostToDevice, sm) != cudaSuccess ||
+      cudaMemsetAsync(c->cs.counters, 0, (batch + 1) * sizeof(uint32_t), sm) != cudaSuccess ||
+      cudaMemsetAsync(c->err, 0, sizeof(int32_t), sm) != cudaSuccess) {
     set_last_error("initial copies failed");
     return fail(DG_ERR_CUDA);
   }
-  dg::launch_init_canvas(c);
+  dg::launch_init_canvas(c->ex, c->cs, c->B, c->C, model->vocab);
   st = check_launch("init canvas");
   if (st != DG_OK) return fail(st);
-  if (cudaStreamSynchronize(c->stream) != cudaSuccess) {
+  if (cudaStreamSynchronize(sm) != cudaSuccess) {
     set_last_error("init synchronize failed");
     return fail(DG_ERR_CUDA);
   }
@@ -272,7 +345,17 @@ dg_status dg_denoise_step(dg_ctx* ctx, const dg_schedule* sched, const dg_step_o
   DG_ARG(ctx != nullptr, "ctx is NULL");
   dg_status st = validate_sched(sched);
   if (st != DG_OK) return st;
-  return enqueue_step(ctx, *sched, dbg);
+  if (dbg) return enqueue_step(ctx, *sched, dbg);
+  return launch_step_graph(ctx, *sched);
+}
+
+dg_status dg_canvas_reset(dg_ctx* ctx, const uint64_t* seeds) {
+  DG_ARG(ctx != nullptr, "ctx is NULL");
+  if (seeds)
+    DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.seed, seeds, ctx->B * sizeof(uint64_t), cudaMemcpyHostToDevice,
+                                ctx->ex.stream));
+  dg::launch_init_canvas(ctx->ex, ctx->cs, ctx->B, ctx->C, ctx->m.vocab);
+  return check_launch("reset canvas");
 }
 
 dg_status dg_decode_block(dg_ctx* ctx, const dg_schedule* sched, int32_t* tokens_out, int32_t* steps_out) {
@@ -283,38 +366,38 @@ dg_status dg_decode_block(dg_ctx* ctx, const dg_schedule* sched, int32_t* tokens
   // remaining positions at the last step), so max_steps launches suffice; the
   // device flag lets the host stop early without a per-step round trip.
   int32_t all = 0;
-  DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->stream));
-  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->cs.all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
   int launched = 0;
   while (!all && launched < sched->max_steps) {
     const int batch = std::min(4, sched->max_steps - launched);
     for (int i = 0; i < batch; ++i) {
-      st = enqueue_step(ctx, *sched, nullptr);
+      st = launch_step_graph(ctx, *sched);
       if (st != DG_OK) return st;
     }
     launched += batch;
-    DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->stream));
-    DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+    DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->cs.all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->ex.stream));
+    DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
   }
   st = read_device_error(ctx);
   if (st != DG_OK) return st;
   if (tokens_out)
-    DG_CUDA_RET(cudaMemcpyAsync(tokens_out, ctx->tok, ctx->M * sizeof(int32_t), cudaMemcpyDefault, ctx->stream));
+    DG_CUDA_RET(cudaMemcpyAsync(tokens_out, ctx->cs.tok, ctx->M * sizeof(int32_t), cudaMemcpyDefault, ctx->ex.stream));
   if (steps_out)
-    DG_CUDA_RET(cudaMemcpyAsync(steps_out, ctx->step, ctx->B * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->stream));
-  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+    DG_CUDA_RET(cudaMemcpyAsync(steps_out, ctx->cs.step, ctx->B * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
   return DG_OK;
 }
 
 dg_status dg_canvas_get_state(dg_ctx* ctx, dg_state* h) {
   DG_ARG(ctx && h, "NULL argument");
   DG_ARG(h->tokens && h->frozen && h->step && h->seed && h->done, "a state array is NULL");
-  DG_CUDA_RET(cudaMemcpyAsync(h->tokens, ctx->tok, ctx->M * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(h->frozen, ctx->frozen, ctx->M, cudaMemcpyDeviceToHost, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(h->step, ctx->step, ctx->B * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(h->seed, ctx->seed, ctx->B * sizeof(uint64_t), cudaMemcpyDeviceToHost, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(h->done, ctx->done, ctx->B, cudaMemcpyDeviceToHost, ctx->stream));
-  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->tokens, ctx->cs.tok, ctx->M * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->frozen, ctx->cs.frozen, ctx->M, cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->step, ctx->cs.step, ctx->B * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->seed, ctx->cs.seed, ctx->B * sizeof(uint64_t), cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(h->done, ctx->cs.done, ctx->B, cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
   return read_device_error(ctx);
 }
 
@@ -327,14 +410,31 @@ dg_status dg_canvas_set_state(dg_ctx* ctx, const dg_state* h) {
     DG_ARG(h->step[b] >= 0, "negative step");
     all &= h->done[b] ? 1 : 0;
   }
-  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(ctx->tok, h->tokens, ctx->M * sizeof(int32_t), cudaMemcpyHostToDevice, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(ctx->frozen, h->frozen, ctx->M, cudaMemcpyHostToDevice, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(ctx->step, h->step, ctx->B * sizeof(int32_t), cudaMemcpyHostToDevice, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(ctx->seed, h->seed, ctx->B * sizeof(uint64_t), cudaMemcpyHostToDevice, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(ctx->done, h->done, ctx->B, cudaMemcpyHostToDevice, ctx->stream));
-  DG_CUDA_RET(cudaMemcpyAsync(ctx->all_done, &all, sizeof(int32_t), cudaMemcpyHostToDevice, ctx->stream));
-  DG_CUDA_RET(cudaStreamSynchronize(ctx->stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.tok, h->tokens, ctx->M * sizeof(int32_t), cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.frozen, h->frozen, ctx->M, cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.step, h->step, ctx->B * sizeof(int32_t), cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.seed, h->seed, ctx->B * sizeof(uint64_t), cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.done, h->done, ctx->B, cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.all_done, &all, sizeof(int32_t), cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
+  return DG_OK;
+}
+
+dg_status dg_canvas_set_timing_events(dg_ctx* ctx, int32_t n, void* const* starts, void* const* stops) {
+  DG_ARG(ctx != nullptr, "ctx is NULL");
+  DG_ARG(n >= 0 && n <= 64, "n must be in [0, 64]");
+  if (n > 0) DG_ARG(starts && stops, "event arrays are NULL");
+  for (int i = 0; i < n; ++i) DG_ARG(starts[i] && stops[i], "NULL event");
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
+  drop_graphs(ctx);
+  ctx->ev_start.clear();
+  ctx->ev_stop.clear();
+  for (int i = 0; i < n; ++i) {
+    ctx->ev_start.push_back(static_cast<cudaEvent_t>(starts[i]));
+    ctx->ev_stop.push_back(static_cast<cudaEvent_t>(stops[i]));
+  }
+  ctx->step_launch_count = 0;
   return DG_OK;
 }
 
@@ -346,10 +446,11 @@ dg_status dg_canvas_sync(dg_ctx* ctx) {
 void dg_canvas_destroy(dg_ctx* ctx) {
   if (!ctx) return;
   if (ctx->ws) {
-    cudaStreamSynchronize(ctx->stream);
+    cudaStreamSynchronize(ctx->ex.stream);
     cudaFree(ctx->ws);
   }
-  if (ctx->graph_exec) cudaGraphExecDestroy(ctx->graph_exec);
+  drop_graphs(ctx);
+  if (ctx->capture_stream) cudaStreamDestroy(ctx->capture_stream);
   delete ctx;
 }
 

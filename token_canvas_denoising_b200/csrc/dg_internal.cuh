@@ -1,6 +1,8 @@
 // Internal declarations of libdgcanvas: the context, its workspace layout and
 // the kernel launchers. Not part of the C ABI.
 #pragma once
+#include <cuda.h>
+
 #include <string>
 #include <vector>
 
@@ -32,12 +34,52 @@ struct LmPartials {
   int P;
 };
 
-// Split-KV attention partials: unnormalised O plus (max, sum) per query row.
-struct AttnPartials {
-  float* o;      // [splits][M*Hq][h]
-  float* ml;     // [splits][M*Hq][2]
-  int splits;
+// Where and how kernels are launched.
+struct Exec {
+  cudaStream_t stream = nullptr;
+  int* err = nullptr;   // device error word
+  int launches = 0;     // kernels queued (for launch accounting)
+  int sm_count = 148;
 };
+
+// Shapes of one attention call.
+struct AttnShape {
+  int B, C, Hq, Hk, h;
+};
+
+void set_last_error(const std::string& msg);
+
+// ---- embed / linear / attention / LM head (dtype-dispatched)
+void launch_embed(Exec& ex, int dtype, const void* E, const int32_t* tok, void* X, int M, int d, int V);
+void launch_linear_simple(Exec& ex, int dtype, const void* A, const void* W, const void* R, void* out,
+                          int M, int N, int K);
+void launch_attention_simple(Exec& ex, int dtype, const void* Q, const PrefixDesc* d_prefix, const void* Kc,
+                             const void* Vc, void* O, const AttnShape& s);
+void launch_lmhead_simple(Exec& ex, int dtype, const void* hs, const void* W, const float* invT,
+                          LmPartials part, int M, int d, int V);
+
+// tcgen05 LM head (bf16): vocab partitions for M rows, tensor maps, launch
+int lmhead_tc_partitions(int M, int V, int sm_count);
+bool lmhead_tc_prepare(const void* hs, const void* lm_head, int M, int d, int V, CUtensorMap* tmA,
+                       CUtensorMap* tmB);
+void launch_lmhead_tc(Exec& ex, const CUtensorMap& tmA, const CUtensorMap& tmB, LmPartials part,
+                      const float* invT, int M, int d, int V);
+
+// ---- canvas bookkeeping
+struct CanvasState {
+  int32_t* tok;
+  uint8_t* frozen;
+  int32_t* step;
+  uint64_t* seed;
+  uint8_t* done;
+  int32_t* all_done;
+  uint32_t* counters;  // [B + 1], zero between launches
+};
+void launch_init_canvas(Exec& ex, const CanvasState& cs, int B, int C, int V);
+// Merge the LM-head partials into ent/am; with `sched` non-null also run the
+// freeze / stop / re-noise selection on every canvas.
+void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uint8_t* fmask,
+                         const CanvasState* cs, const dg_schedule* sched, int B, int C, int V);
 
 }  // namespace dg
 
@@ -49,21 +91,14 @@ struct dg_ctx {
   std::vector<const void*> pk, pv;
   int max_S = 0;
   const float* inv_temp = nullptr;
-  cudaStream_t stream = nullptr;
-  int device = 0, sm_count = 0;
+  int device = 0;
+  dg::Exec ex;
 
   void* ws = nullptr;
   size_t ws_bytes = 0;
 
-  // decode state
-  int32_t* tok = nullptr;
-  uint8_t* frozen = nullptr;
-  int32_t* step = nullptr;
-  uint64_t* seed = nullptr;
-  uint8_t* done = nullptr;
-  int32_t* err = nullptr;        // device error word
-  int32_t* all_done = nullptr;   // 1 when every canvas is done
-  uint32_t* counters = nullptr;  // scratch arrival counters (zero between launches)
+  dg::CanvasState cs{};
+  int32_t* err = nullptr;
 
   // activations, storage dtype
   void *X = nullptr, *Q = nullptr, *Kc = nullptr, *Vc = nullptr, *O = nullptr;
@@ -71,33 +106,21 @@ struct dg_ctx {
   dg::PrefixDesc* d_prefix = nullptr;
 
   dg::LmPartials lm{};
-  dg::AttnPartials attn{};
   float* ent = nullptr;
   int32_t* am = nullptr;
-  uint8_t* fmask = nullptr;
+
+  // tensor maps (bf16 path)
+  CUtensorMap tm_lm_a, tm_lm_b;
 
   int launches = 0;  // kernels queued by the last denoise step
 
-  // captured step graph
-  cudaGraphExec_t graph_exec = nullptr;
+  // the step captured as CUDA graphs (per schedule), launched on ex.stream;
+  // with timing events there is one graph variant per event pair, used in turn
+  cudaStream_t capture_stream = nullptr;
+  std::vector<cudaGraphExec_t> graphs;
   dg_schedule graph_sched{};
-  bool graph_valid = false;
+  int graph_launches = 0;
+  std::vector<cudaEvent_t> ev_start, ev_stop;
+  cudaEvent_t cur_ev_start = nullptr, cur_ev_stop = nullptr;  // set while capturing
+  long long step_launch_count = 0;
 };
-
-namespace dg {
-
-// error reporting (thread-local message)
-void set_last_error(const std::string& msg);
-
-// simple CUDA-core kernels (f32 storage)
-void launch_embed(dg_ctx* c);
-void launch_linear_simple(dg_ctx* c, const void* A, const void* W, const void* R, void* out,
-                          int M, int N, int K);
-void launch_attention_simple(dg_ctx* c);
-void launch_lmhead_simple(dg_ctx* c, const void* hs);
-
-// canvas bookkeeping
-void launch_init_canvas(dg_ctx* c);
-void launch_merge_select(dg_ctx* c, const dg_schedule& s, uint8_t* fmask_out);
-
-}  // namespace dg

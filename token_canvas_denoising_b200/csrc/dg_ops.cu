@@ -1,0 +1,118 @@
+// Single-operation entry points (include/dg_ops.h): the step's kernels on
+// caller buffers, each with its own stream-ordered temporaries.
+#include <string>
+#include <vector>
+
+#include "dg_internal.cuh"
+#include "dg_ops.h"
+
+using dg::set_last_error;
+
+namespace {
+
+#define OP_ARG(cond, msg)                                          \
+  do {                                                             \
+    if (!(cond)) {                                                 \
+      set_last_error(std::string("invalid argument: ") + (msg));   \
+      return DG_ERR_INVALID_ARG;                                   \
+    }                                                              \
+  } while (0)
+#define OP_UNSUP(cond, msg)                                        \
+  do {                                                             \
+    if (!(cond)) {                                                 \
+      set_last_error(std::string("unsupported: ") + (msg));        \
+      return DG_ERR_UNSUPPORTED;                                   \
+    }                                                              \
+  } while (0)
+
+dg_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return DG_OK;
+  set_last_error(std::string(what) + ": " + cudaGetErrorString(e));
+  return e == cudaErrorMemoryAllocation ? DG_ERR_OOM : DG_ERR_CUDA;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dg::Exec make_exec(void* stream) {
+  dg::Exec ex;
+  ex.stream = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&ex.sm_count, cudaDevAttrMultiProcessorCount, dev);
+  return ex;
+}
+
+}  // namespace
+
+extern "C" {
+
+dg_status dg_lmhead_entropy(int32_t dtype, const void* hs, const void* lm_head, const float* inv_temp, int32_t M,
+                            int32_t d, int32_t V, float* ent, int32_t* argmax, void* stream) {
+  OP_ARG(dtype == DG_F32 || dtype == DG_BF16, "dtype");
+  OP_ARG(hs && lm_head && ent && argmax, "NULL buffer");
+  OP_ARG(M >= 1 && d >= 1 && V >= 2, "sizes");
+  OP_ARG(al16(hs) && al16(lm_head), "hs / lm_head must be 16-byte aligned");
+  OP_UNSUP(d % 8 == 0, "d % 8 != 0");
+  if (dtype == DG_BF16) OP_UNSUP(d % 64 == 0 && V % 256 == 0, "bf16 needs d % 64 == 0 and V % 256 == 0");
+  dg::Exec ex = make_exec(stream);
+  dg::LmPartials part;
+  part.P = dtype == DG_BF16 ? dg::lmhead_tc_partitions(M, V, ex.sm_count) : std::max(1, std::min(128, V / 1024));
+  dg_status st = cuda_status(cudaMallocAsync((void**)&part.rec, sizeof(dg::LmRec) * (size_t)M * part.P, ex.stream),
+                             "cudaMallocAsync");
+  if (st != DG_OK) return st;
+  if (dtype == DG_BF16) {
+    CUtensorMap a, b;
+    if (!dg::lmhead_tc_prepare(hs, lm_head, M, d, V, &a, &b)) {
+      cudaFreeAsync(part.rec, ex.stream);
+      return DG_ERR_CUDA;
+    }
+    dg::launch_lmhead_tc(ex, a, b, part, inv_temp, M, d, V);
+  } else {
+    dg::launch_lmhead_simple(ex, dtype, hs, lm_head, inv_temp, part, M, d, V);
+  }
+  dg::launch_merge_select(ex, part, ent, argmax, nullptr, nullptr, nullptr, 1, M, V);
+  st = cuda_status(cudaGetLastError(), "launch");
+  cudaFreeAsync(part.rec, ex.stream);
+  return st;
+}
+
+dg_status dg_attention(int32_t dtype, const void* q, const void* kc, const void* vc, int32_t B, int32_t C,
+                       int32_t Hq, int32_t Hk, int32_t h, const int32_t* prefix_len, const void* const* prefix_k,
+                       const void* const* prefix_v, void* o, void* stream) {
+  OP_ARG(dtype == DG_F32 || dtype == DG_BF16, "dtype");
+  OP_ARG(q && kc && vc && o && prefix_len, "NULL buffer");
+  OP_ARG(B >= 1 && C >= 1 && Hq >= 1 && Hk >= 1 && Hq % Hk == 0, "sizes");
+  if (dtype == DG_BF16) OP_UNSUP(h == 128, "bf16 needs h == 128");
+  else OP_UNSUP(h % 32 == 0 && h <= 128, "f32 needs h in {32, 64, 96, 128}");
+  std::vector<dg::PrefixDesc> pd(B);
+  for (int b = 0; b < B; ++b) {
+    OP_ARG(prefix_len[b] >= 0, "negative prefix length");
+    if (prefix_len[b] > 0) OP_ARG(prefix_k && prefix_v && prefix_k[b] && prefix_v[b], "NULL prefix pointer");
+    pd[b] = {prefix_len[b] ? prefix_k[b] : nullptr, prefix_len[b] ? prefix_v[b] : nullptr, prefix_len[b], 0};
+  }
+  dg::Exec ex = make_exec(stream);
+  dg::PrefixDesc* dpd = nullptr;
+  dg_status st = cuda_status(cudaMallocAsync((void**)&dpd, sizeof(dg::PrefixDesc) * B, ex.stream), "cudaMallocAsync");
+  if (st != DG_OK) return st;
+  st = cuda_status(cudaMemcpyAsync(dpd, pd.data(), sizeof(dg::PrefixDesc) * B, cudaMemcpyHostToDevice, ex.stream),
+                   "cudaMemcpyAsync");
+  if (st == DG_OK) {
+    dg::AttnShape sh{B, C, Hq, Hk, h};
+    dg::launch_attention_simple(ex, dtype, q, dpd, kc, vc, o, sh);
+    st = cuda_status(cudaGetLastError(), "launch");
+  }
+  cudaFreeAsync(dpd, ex.stream);
+  return st;
+}
+
+dg_status dg_linear(int32_t dtype, const void* a, const void* w, const void* residual, void* out, int32_t M,
+                    int32_t N, int32_t K, void* stream) {
+  OP_ARG(dtype == DG_F32 || dtype == DG_BF16, "dtype");
+  OP_ARG(a && w && out, "NULL buffer");
+  OP_ARG(M >= 1 && N >= 1 && K >= 1, "sizes");
+  dg::Exec ex = make_exec(stream);
+  dg::launch_linear_simple(ex, dtype, a, w, residual, out, M, N, K);
+  return cuda_status(cudaGetLastError(), "launch");
+}
+
+}  // extern "C"

@@ -27,9 +27,9 @@ __global__ void init_canvas_kernel(int32_t* tok, uint8_t* frozen, int32_t* step,
   }
 }
 
-void launch_init_canvas(dg_ctx* c) {
-  init_canvas_kernel<<<c->B, 256, 0, c->stream>>>(c->tok, c->frozen, c->step, c->seed, c->done,
-                                                 c->all_done, c->C, c->m.vocab);
+void launch_init_canvas(Exec& ex, const CanvasState& cs, int B, int C, int V) {
+  init_canvas_kernel<<<B, 256, 0, ex.stream>>>(cs.tok, cs.frozen, cs.step, cs.seed, cs.done, cs.all_done, C, V);
+  ex.launches++;
 }
 
 // ------------------------------------------------------------------ merge + select
@@ -48,6 +48,7 @@ struct SelectArgs {
   int32_t* err;
   int B, C, V, max_steps, adaptive;
   float stop_entropy;
+  int select;           // 0: only merge the partials into ent / am
 };
 
 __device__ __forceinline__ EntStats load_rec(const LmRec* r) {
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
       a.am[r] = st.idx;
     }
   }
+  if (!a.select) return;
   // ---- arrival: the last block of canvas b runs the selection
   __shared__ int s_last;
   __syncthreads();
@@ -172,29 +174,33 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
   }
 }
 
-void launch_merge_select(dg_ctx* c, const dg_schedule& s, uint8_t* fmask_out) {
-  SelectArgs a;
-  a.part = c->lm;
-  a.ent = c->ent;
-  a.am = c->am;
-  a.fmask = fmask_out;
-  a.tok = c->tok;
-  a.frozen = c->frozen;
-  a.step = c->step;
-  a.seed = c->seed;
-  a.done = c->done;
-  a.all_done = c->all_done;
-  a.counters = c->counters;
-  a.err = c->err;
-  a.B = c->B;
-  a.C = c->C;
-  a.V = c->m.vocab;
-  a.max_steps = s.max_steps;
-  a.adaptive = s.adaptive_stop;
-  a.stop_entropy = s.stop_entropy;
-  dim3 grid(ceil_div(c->C, 8), c->B);
-  merge_select_kernel<<<grid, 256, 0, c->stream>>>(a);
-  c->launches++;
+void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uint8_t* fmask,
+                         const CanvasState* cs, const dg_schedule* sched, int B, int C, int V) {
+  SelectArgs a{};
+  a.part = part;
+  a.ent = ent;
+  a.am = am;
+  a.fmask = fmask;
+  a.err = ex.err;
+  a.B = B;
+  a.C = C;
+  a.V = V;
+  a.select = (cs && sched) ? 1 : 0;
+  if (a.select) {
+    a.tok = cs->tok;
+    a.frozen = cs->frozen;
+    a.step = cs->step;
+    a.seed = cs->seed;
+    a.done = cs->done;
+    a.all_done = cs->all_done;
+    a.counters = cs->counters;
+    a.max_steps = sched->max_steps;
+    a.adaptive = sched->adaptive_stop;
+    a.stop_entropy = sched->stop_entropy;
+  }
+  dim3 grid(ceil_div(C, 8), B);
+  merge_select_kernel<<<grid, 256, 0, ex.stream>>>(a);
+  ex.launches++;
 }
 
 }  // namespace dg

@@ -23,14 +23,13 @@ __global__ void embed_kernel(const T* __restrict__ E, const int32_t* __restrict_
   for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src[i];
 }
 
-void launch_embed(dg_ctx* c) {
-  const int d = c->m.d_model, V = c->m.vocab;
-  if (c->m.dtype == DG_F32)
-    embed_kernel<float><<<c->M, 128, 0, c->stream>>>((const float*)c->m.embed, c->tok, (float*)c->X, d, V, c->err);
+void launch_embed(Exec& ex, int dtype, const void* E, const int32_t* tok, void* X, int M, int d, int V) {
+  if (dtype == DG_F32)
+    embed_kernel<float><<<M, 128, 0, ex.stream>>>((const float*)E, tok, (float*)X, d, V, ex.err);
   else
-    embed_kernel<__nv_bfloat16><<<c->M, 128, 0, c->stream>>>((const __nv_bfloat16*)c->m.embed, c->tok,
-                                                             (__nv_bfloat16*)c->X, d, V, c->err);
-  c->launches++;
+    embed_kernel<__nv_bfloat16><<<M, 128, 0, ex.stream>>>((const __nv_bfloat16*)E, tok, (__nv_bfloat16*)X, d,
+                                                          V, ex.err);
+  ex.launches++;
 }
 
 // ------------------------------------------------------------------ linear
@@ -71,17 +70,17 @@ __global__ void linear_simple_kernel(const T* __restrict__ A, const T* __restric
   }
 }
 
-void launch_linear_simple(dg_ctx* c, const void* A, const void* W, const void* R, void* out,
+void launch_linear_simple(Exec& ex, int dtype, const void* A, const void* W, const void* R, void* out,
                           int M, int N, int K) {
   dim3 grid(ceil_div(N, 32), ceil_div(M, 32));
-  if (c->m.dtype == DG_F32)
-    linear_simple_kernel<float><<<grid, 256, 0, c->stream>>>((const float*)A, (const float*)W,
+  if (dtype == DG_F32)
+    linear_simple_kernel<float><<<grid, 256, 0, ex.stream>>>((const float*)A, (const float*)W,
                                                              (const float*)R, (float*)out, M, N, K);
   else
-    linear_simple_kernel<__nv_bfloat16><<<grid, 256, 0, c->stream>>>(
+    linear_simple_kernel<__nv_bfloat16><<<grid, 256, 0, ex.stream>>>(
         (const __nv_bfloat16*)A, (const __nv_bfloat16*)W, (const __nv_bfloat16*)R,
         (__nv_bfloat16*)out, M, N, K);
-  c->launches++;
+  ex.launches++;
 }
 
 // ------------------------------------------------------------------ attention
@@ -132,27 +131,28 @@ __global__ void attn_simple_kernel(const T* __restrict__ Q, const PrefixDesc* __
 }
 
 template <typename T>
-static void attn_simple_dispatch(dg_ctx* c) {
-  const int h = c->m.head_dim, Hq = c->m.n_q_heads, Hk = c->m.n_kv_heads;
-  const int warps = c->B * c->C * Hq;
+static void attn_simple_dispatch(Exec& ex, const void* Qv, const PrefixDesc* pre, const void* Kcv,
+                                 const void* Vcv, void* Ov, const AttnShape& sh) {
+  const int warps = sh.B * sh.C * sh.Hq;
   const int blocks = ceil_div(warps, 8);
-  const float scale = 1.f / sqrtf((float)h);
-  const T* Q = (const T*)c->Q;
-  const T* Kc = (const T*)c->Kc;
-  const T* Vc = (const T*)c->Vc;
-  T* O = (T*)c->O;
-  switch (h / 32) {
-    case 1: attn_simple_kernel<T, 1><<<blocks, 256, 0, c->stream>>>(Q, c->d_prefix, Kc, Vc, O, c->B, c->C, Hq, Hk, scale); break;
-    case 2: attn_simple_kernel<T, 2><<<blocks, 256, 0, c->stream>>>(Q, c->d_prefix, Kc, Vc, O, c->B, c->C, Hq, Hk, scale); break;
-    case 3: attn_simple_kernel<T, 3><<<blocks, 256, 0, c->stream>>>(Q, c->d_prefix, Kc, Vc, O, c->B, c->C, Hq, Hk, scale); break;
-    default: attn_simple_kernel<T, 4><<<blocks, 256, 0, c->stream>>>(Q, c->d_prefix, Kc, Vc, O, c->B, c->C, Hq, Hk, scale); break;
+  const float scale = 1.f / sqrtf((float)sh.h);
+  const T* Q = (const T*)Qv;
+  const T* Kc = (const T*)Kcv;
+  const T* Vc = (const T*)Vcv;
+  T* O = (T*)Ov;
+  switch (sh.h / 32) {
+    case 1: attn_simple_kernel<T, 1><<<blocks, 256, 0, ex.stream>>>(Q, pre, Kc, Vc, O, sh.B, sh.C, sh.Hq, sh.Hk, scale); break;
+    case 2: attn_simple_kernel<T, 2><<<blocks, 256, 0, ex.stream>>>(Q, pre, Kc, Vc, O, sh.B, sh.C, sh.Hq, sh.Hk, scale); break;
+    case 3: attn_simple_kernel<T, 3><<<blocks, 256, 0, ex.stream>>>(Q, pre, Kc, Vc, O, sh.B, sh.C, sh.Hq, sh.Hk, scale); break;
+    default: attn_simple_kernel<T, 4><<<blocks, 256, 0, ex.stream>>>(Q, pre, Kc, Vc, O, sh.B, sh.C, sh.Hq, sh.Hk, scale); break;
   }
 }
 
-void launch_attention_simple(dg_ctx* c) {
-  if (c->m.dtype == DG_F32) attn_simple_dispatch<float>(c);
-  else attn_simple_dispatch<__nv_bfloat16>(c);
-  c->launches++;
+void launch_attention_simple(Exec& ex, int dtype, const void* Q, const PrefixDesc* d_prefix, const void* Kc,
+                             const void* Vc, void* O, const AttnShape& s) {
+  if (dtype == DG_F32) attn_simple_dispatch<float>(ex, Q, d_prefix, Kc, Vc, O, s);
+  else attn_simple_dispatch<__nv_bfloat16>(ex, Q, d_prefix, Kc, Vc, O, s);
+  ex.launches++;
 }
 
 // ------------------------------------------------------------------ LM head
@@ -199,18 +199,17 @@ __global__ void lmhead_simple_kernel(const T* __restrict__ Hs, const T* __restri
   }
 }
 
-void launch_lmhead_simple(dg_ctx* c, const void* hs) {
-  const int V = c->m.vocab;
-  const int chunk = ceil_div(V, c->lm.P);
-  dim3 grid(c->lm.P, ceil_div(c->M, 8));
-  if (c->m.dtype == DG_F32)
-    lmhead_simple_kernel<float><<<grid, 256, 0, c->stream>>>((const float*)hs, (const float*)c->m.lm_head,
-                                                             c->inv_temp, c->lm, c->M, c->m.d_model, V, chunk);
+void launch_lmhead_simple(Exec& ex, int dtype, const void* hs, const void* W, const float* invT,
+                          LmPartials part, int M, int d, int V) {
+  const int chunk = ceil_div(V, part.P);
+  dim3 grid(part.P, ceil_div(M, 8));
+  if (dtype == DG_F32)
+    lmhead_simple_kernel<float><<<grid, 256, 0, ex.stream>>>((const float*)hs, (const float*)W, invT, part, M,
+                                                             d, V, chunk);
   else
-    lmhead_simple_kernel<__nv_bfloat16><<<grid, 256, 0, c->stream>>>(
-        (const __nv_bfloat16*)hs, (const __nv_bfloat16*)c->m.lm_head, c->inv_temp, c->lm, c->M,
-        c->m.d_model, V, chunk);
-  c->launches++;
+    lmhead_simple_kernel<__nv_bfloat16><<<grid, 256, 0, ex.stream>>>(
+        (const __nv_bfloat16*)hs, (const __nv_bfloat16*)W, invT, part, M, d, V, chunk);
+  ex.launches++;
 }
 
 }  // namespace dg

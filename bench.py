@@ -305,6 +305,7 @@ def bench_b200(args, rank, world, local_rank):
     # state goes host->device (pinned) and the tokens come back device->host
     e2e = None
     if rank == 0 or world > 1:
+        cv.reset()  # a fresh block: step 0, nothing frozen
         st0 = cv.get_state()
         pin = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for k, v in st0.items()}
         pin_np = {k: v.numpy() for k, v in pin.items()}
@@ -319,6 +320,7 @@ def bench_b200(args, rank, world, local_rank):
             cv.set_state(pin_np)
             _, steps = cv.decode(sched, tok_out)
             total_steps += max(steps)
+            assert max(steps) == cfg.max_steps, steps
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)

@@ -46,7 +46,7 @@ dg_status dg_attention(int32_t dtype, const void *q, const void *kc, const void 
 
 /* out[M][N] = a[M][K] . w[N][K]^T (+ residual[M][N] if not NULL), f32
  * accumulate, one rounding to dtype ([P3] 架构解剖 2: the canvas's K/V are
- * re-projected every step). bf16 needs K % 64 == 0 and N % 16 == 0. */
+ * re-projected every step). bf16 needs K % 64 == 0 and N % 64 == 0. */
 dg_status dg_linear(int32_t dtype, const void *a, const void *w, const void *residual, void *out,
                     int32_t M, int32_t N, int32_t K, void *stream);
 

@@ -82,6 +82,11 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   c->lm.rec = w.take<dg::LmRec>(M * (size_t)c->lm.P);
   c->ent = w.take<float>(M);
   c->am = w.take<int32_t>(M);
+  if (c->m.dtype == DG_BF16 && c->attn_splits > 1) {
+    const size_t rows = M * (size_t)c->m.n_q_heads;
+    c->attn.part_o = w.take<float>((size_t)c->attn_splits * rows * 128);
+    c->attn.part_ml = w.take<float>((size_t)c->attn_splits * rows * 2);
+  }
   *total = w.off + 256;
 }
 
@@ -138,12 +143,22 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
   dg::Exec& ex = c->ex;
   ex.launches = 0;
   dg::launch_embed(ex, dt, c->m.embed, c->cs.tok, c->X, M, d, V);
-  dg::launch_linear_simple(ex, dt, c->X, c->m.wq, nullptr, c->Q, M, qd, d);
-  dg::launch_linear_simple(ex, dt, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
-  dg::launch_linear_simple(ex, dt, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
+  if (dt == DG_BF16) {
+    dg::launch_gemm_tc(ex, c->g_qkv, nullptr);
+  } else {
+    dg::launch_linear_simple(ex, dt, c->X, c->m.wq, nullptr, c->Q, M, qd, d);
+    dg::launch_linear_simple(ex, dt, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
+    dg::launch_linear_simple(ex, dt, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
+  }
   dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
-  dg::launch_attention_simple(ex, dt, c->Q, c->d_prefix, c->Kc, c->Vc, c->O, sh);
-  dg::launch_linear_simple(ex, dt, c->O, c->m.wo, c->X, c->Hs, M, d, qd);
+  if (dt == DG_BF16)
+    dg::launch_attn_tc(ex, c->attn);
+  else
+    dg::launch_attention_simple(ex, dt, c->Q, c->d_prefix, c->Kc, c->Vc, c->O, sh);
+  if (dt == DG_BF16)
+    dg::launch_gemm_tc(ex, c->g_wo, c->X);
+  else
+    dg::launch_linear_simple(ex, dt, c->O, c->m.wo, c->X, c->Hs, M, d, qd);
   const void* hs = c->Hs;
   // inside a stream capture, only an "external" record becomes an event node
   if (c->cur_ev_start) DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start, ex.stream, cudaEventRecordExternal));
@@ -295,8 +310,10 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
     set_last_error("no usable CUDA device");
     return fail(DG_ERR_CUDA);
   }
-  if (model->dtype == DG_BF16)
+  if (model->dtype == DG_BF16) {
     c->lm.P = dg::lmhead_tc_partitions(c->M, model->vocab, c->ex.sm_count);
+    c->attn_splits = dg::attn_tc_splits(batch, canvas_len, model->n_q_heads, c->S.data(), c->ex.sm_count);
+  }
   else
     c->lm.P = std::max(1, std::min(128, model->vocab / 1024));
 
@@ -315,9 +332,24 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   c->ws_bytes = total;
   layout_workspace(c, c->ws, &total);
   c->ex.err = c->err;
-  if (model->dtype == DG_BF16 &&
-      !dg::lmhead_tc_prepare(c->Hs, model->lm_head, c->M, model->d_model, model->vocab, &c->tm_lm_a, &c->tm_lm_b))
-    return fail(DG_ERR_CUDA);
+  if (model->dtype == DG_BF16) {
+    const int qd = model->n_q_heads * model->head_dim, kd = model->n_kv_heads * model->head_dim;
+    const void* wqkv[3] = {model->wq, model->wk, model->wv};
+    void* oqkv[3] = {c->Q, c->Kc, c->Vc};
+    const int nqkv[3] = {qd, kd, kd};
+    const void* wo[1] = {model->wo};
+    void* oo[1] = {c->Hs};
+    const int no[1] = {model->d_model};
+    if (!dg::lmhead_tc_prepare(c->Hs, model->lm_head, c->M, model->d_model, model->vocab, &c->tm_lm_a,
+                               &c->tm_lm_b) ||
+        !dg::gemm_tc_prepare(&c->g_qkv, c->X, c->M, model->d_model, 3, wqkv, oqkv, nqkv) ||
+        !dg::gemm_tc_prepare(&c->g_wo, c->O, c->M, qd, 1, wo, oo, no))
+      return fail(DG_ERR_CUDA);
+    dg::AttnShape sh{batch, canvas_len, model->n_q_heads, model->n_kv_heads, model->head_dim};
+    if (!dg::attn_tc_prepare(&c->attn, sh, c->Q, c->Kc, c->Vc, c->S.data(), c->pk.data(), c->pv.data(), c->O,
+                             c->attn.part_o, c->attn.part_ml, c->attn_splits))
+      return fail(DG_ERR_CUDA);
+  }
 
   std::vector<dg::PrefixDesc> pd(batch);
   for (int b = 0; b < batch; ++b) pd[b] = {c->pk[b], c->pv[b], c->S[b], 0};

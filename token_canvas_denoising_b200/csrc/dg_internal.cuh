@@ -65,6 +65,39 @@ bool lmhead_tc_prepare(const void* hs, const void* lm_head, int M, int d, int V,
 void launch_lmhead_tc(Exec& ex, const CUtensorMap& tmA, const CUtensorMap& tmB, LmPartials part,
                       const float* invT, int M, int d, int V);
 
+// tcgen05 projection GEMM (bf16): out_i = A W_i^T (+ R) for up to 3 output
+// segments sharing A; prepared once (tensor maps), launched many times.
+struct alignas(64) GemmTc {
+  unsigned char maps[4 * 128];  // CUtensorMap for A and each W_i
+  int M = 0, K = 0, nseg = 0, tiles = 0;
+  void* out[3] = {nullptr, nullptr, nullptr};
+  int N[3] = {0, 0, 0};
+};
+bool gemm_tc_prepare(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W, void* const* out,
+                     const int* N);
+void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual);
+
+// tcgen05 attention (bf16, head_dim 128): tensor maps per group of up to 8
+// requests, split-KV partial buffers.
+struct AttnTc {
+  struct Group {
+    alignas(64) unsigned char maps[19 * 128];
+    int b0 = 0, nreq = 0;
+    int S[8] = {0};
+  };
+  AttnShape sh{};
+  void* O = nullptr;
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  int splits = 1;
+  std::vector<Group> groups;
+};
+int attn_tc_splits(int B, int C, int Hq, const int* S, int sm_count);
+bool attn_tc_prepare(AttnTc* at, const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
+                     const int32_t* S, const void* const* pk, const void* const* pv, void* O, float* part_o,
+                     float* part_ml, int splits);
+void launch_attn_tc(Exec& ex, const AttnTc& at);
+
 // ---- canvas bookkeeping
 struct CanvasState {
   int32_t* tok;
@@ -111,6 +144,9 @@ struct dg_ctx {
 
   // tensor maps (bf16 path)
   CUtensorMap tm_lm_a, tm_lm_b;
+  dg::GemmTc g_qkv, g_wo;
+  dg::AttnTc attn;
+  int attn_splits = 1;
 
   int launches = 0;  // kernels queued by the last denoise step
 

@@ -91,6 +91,29 @@ dg_status dg_attention(int32_t dtype, const void* q, const void* kc, const void*
     pd[b] = {prefix_len[b] ? prefix_k[b] : nullptr, prefix_len[b] ? prefix_v[b] : nullptr, prefix_len[b], 0};
   }
   dg::Exec ex = make_exec(stream);
+  if (dtype == DG_BF16) {
+    OP_ARG(al16(q) && al16(kc) && al16(vc) && al16(o), "buffers must be 16-byte aligned");
+    dg::AttnShape sh{B, C, Hq, Hk, h};
+    const int splits = dg::attn_tc_splits(B, C, Hq, prefix_len, ex.sm_count);
+    float* part = nullptr;
+    const size_t rows = (size_t)B * C * Hq;
+    if (splits > 1) {
+      dg_status st = cuda_status(cudaMallocAsync((void**)&part, splits * rows * 130 * sizeof(float), ex.stream),
+                                 "cudaMallocAsync");
+      if (st != DG_OK) return st;
+    }
+    dg::AttnTc at;
+    dg_status st = DG_OK;
+    if (!dg::attn_tc_prepare(&at, sh, q, kc, vc, prefix_len, prefix_k, prefix_v, o, part,
+                             part ? part + splits * rows * 128 : nullptr, splits))
+      st = DG_ERR_CUDA;
+    else {
+      dg::launch_attn_tc(ex, at);
+      st = cuda_status(cudaGetLastError(), "launch");
+    }
+    if (part) cudaFreeAsync(part, ex.stream);
+    return st;
+  }
   dg::PrefixDesc* dpd = nullptr;
   dg_status st = cuda_status(cudaMallocAsync((void**)&dpd, sizeof(dg::PrefixDesc) * B, ex.stream), "cudaMallocAsync");
   if (st != DG_OK) return st;
@@ -111,7 +134,18 @@ dg_status dg_linear(int32_t dtype, const void* a, const void* w, const void* res
   OP_ARG(a && w && out, "NULL buffer");
   OP_ARG(M >= 1 && N >= 1 && K >= 1, "sizes");
   dg::Exec ex = make_exec(stream);
-  dg::launch_linear_simple(ex, dtype, a, w, residual, out, M, N, K);
+  if (dtype == DG_BF16) {
+    OP_UNSUP(K % 64 == 0 && N % 64 == 0, "bf16 needs K % 64 == 0 and N % 64 == 0");
+    OP_ARG(al16(a) && al16(w) && al16(out) && (!residual || al16(residual)), "buffers must be 16-byte aligned");
+    dg::GemmTc g;
+    const void* ws[1] = {w};
+    void* os[1] = {out};
+    const int ns[1] = {N};
+    if (!dg::gemm_tc_prepare(&g, a, M, K, 1, ws, os, ns)) return DG_ERR_CUDA;
+    dg::launch_gemm_tc(ex, g, residual);
+  } else {
+    dg::launch_linear_simple(ex, dtype, a, w, residual, out, M, N, K);
+  }
   return cuda_status(cudaGetLastError(), "launch");
 }
 

@@ -82,6 +82,12 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   c->lm.rec = w.take<dg::LmRec>(M * (size_t)c->lm.P);
   c->ent = w.take<float>(M);
   c->am = w.take<int32_t>(M);
+  if (c->m.dtype == DG_BF16) {
+    c->g_qkv.part = w.take<float>(dg::gemm_tc_partial_floats(c->g_qkv));
+    c->g_qkv.counters = w.take<unsigned>(dg::gemm_tc_counters(c->g_qkv));
+    c->g_wo.part = w.take<float>(dg::gemm_tc_partial_floats(c->g_wo));
+    c->g_wo.counters = w.take<unsigned>(dg::gemm_tc_counters(c->g_wo));
+  }
   if (c->m.dtype == DG_BF16 && c->attn_splits > 1) {
     const size_t rows = M * (size_t)c->m.n_q_heads;
     c->attn.part_o = w.take<float>((size_t)c->attn_splits * rows * 128);
@@ -313,6 +319,16 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   if (model->dtype == DG_BF16) {
     c->lm.P = dg::lmhead_tc_partitions(c->M, model->vocab, c->ex.sm_count);
     c->attn_splits = dg::attn_tc_splits(batch, canvas_len, model->n_q_heads, c->S.data(), c->ex.sm_count);
+    // tile / split choice only (buffers are bound after the workspace exists)
+    const int qd = model->n_q_heads * model->head_dim, kd = model->n_kv_heads * model->head_dim;
+    const void* wqkv[3] = {model->wq, model->wk, model->wv};
+    void* none[3] = {nullptr, nullptr, nullptr};
+    const int nqkv[3] = {qd, kd, kd};
+    const void* wo[1] = {model->wo};
+    const int no[1] = {model->d_model};
+    if (!dg::gemm_tc_prepare(&c->g_qkv, model->embed, c->M, model->d_model, 3, wqkv, none, nqkv, c->ex.sm_count) ||
+        !dg::gemm_tc_prepare(&c->g_wo, model->embed, c->M, qd, 1, wo, none, no, c->ex.sm_count))
+      return fail(DG_ERR_CUDA);
   }
   else
     c->lm.P = std::max(1, std::min(128, model->vocab / 1024));
@@ -340,10 +356,21 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
     const void* wo[1] = {model->wo};
     void* oo[1] = {c->Hs};
     const int no[1] = {model->d_model};
+    dg::GemmTc gq = c->g_qkv, gw = c->g_wo;  // keep the bound buffers
     if (!dg::lmhead_tc_prepare(c->Hs, model->lm_head, c->M, model->d_model, model->vocab, &c->tm_lm_a,
                                &c->tm_lm_b) ||
-        !dg::gemm_tc_prepare(&c->g_qkv, c->X, c->M, model->d_model, 3, wqkv, oqkv, nqkv) ||
-        !dg::gemm_tc_prepare(&c->g_wo, c->O, c->M, qd, 1, wo, oo, no))
+        !dg::gemm_tc_prepare(&c->g_qkv, c->X, c->M, model->d_model, 3, wqkv, oqkv, nqkv, c->ex.sm_count) ||
+        !dg::gemm_tc_prepare(&c->g_wo, c->O, c->M, qd, 1, wo, oo, no, c->ex.sm_count))
+      return fail(DG_ERR_CUDA);
+    c->g_qkv.part = gq.part;
+    c->g_qkv.counters = gq.counters;
+    c->g_wo.part = gw.part;
+    c->g_wo.counters = gw.counters;
+    if (c->g_qkv.counters &&
+        cudaMemsetAsync(c->g_qkv.counters, 0, dg::gemm_tc_counters(c->g_qkv) * sizeof(unsigned), c->ex.stream) != cudaSuccess)
+      return fail(DG_ERR_CUDA);
+    if (c->g_wo.counters &&
+        cudaMemsetAsync(c->g_wo.counters, 0, dg::gemm_tc_counters(c->g_wo) * sizeof(unsigned), c->ex.stream) != cudaSuccess)
       return fail(DG_ERR_CUDA);
     dg::AttnShape sh{batch, canvas_len, model->n_q_heads, model->n_kv_heads, model->head_dim};
     if (!dg::attn_tc_prepare(&c->attn, sh, c->Q, c->Kc, c->Vc, c->S.data(), c->pk.data(), c->pv.data(), c->O,

@@ -98,16 +98,15 @@ struct EntStats {
 
 __device__ __forceinline__ EntStats ent_empty() { return {-INFINITY, 0.f, 0.f, -INFINITY, 0x7fffffff}; }
 
-// Merge two partial states; `a` covers lower vocab ids than `b` when their
-// argmax values tie, so ties resolve to the lower id either way.
+// Merge two partial states; argmax ties resolve to the lower vocab id.
 __device__ __forceinline__ EntStats ent_merge(EntStats a, EntStats b) {
   EntStats r;
   float m = fmaxf(a.m, b.m);
   if (m == -INFINITY) {
     r.m = m; r.z = 0.f; r.s = 0.f;
   } else {
-    float ea = (a.m == -INFINITY) ? 0.f : expf(a.m - m);
-    float eb = (b.m == -INFINITY) ? 0.f : expf(b.m - m);
+    float ea = (a.m == -INFINITY) ? 0.f : __expf(a.m - m);
+    float eb = (b.m == -INFINITY) ? 0.f : __expf(b.m - m);
     // S relative to the new maximum: e^(m_i - m) * (S_i + (m_i - m) Z_i)
     float sa = (a.m == -INFINITY) ? 0.f : ea * (a.s + (a.m - m) * a.z);
     float sb = (b.m == -INFINITY) ? 0.f : eb * (b.s + (b.m - m) * b.z);

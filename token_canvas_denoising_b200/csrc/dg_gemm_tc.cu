@@ -4,11 +4,18 @@
 // K/V are recomputed every step, "DiffusionGemma深度拆解：从逐字蹦到整块喷，LLM生成范式
 // 的结构性跃迁", 架构解剖 2) and for the output projection with the residual.
 //
-// CTA tile: up to 256 rows (two 128-row halves) x 64 output columns, full K.
-// K-loop of 64-wide blocks through a 5-stage TMA pipeline (A 32 KB + B 8 KB per
-// stage). Warp 0 issues TMA, warp 1 allocates TMEM and issues the MMAs
-// (M=128, N=64, K=16) into two accumulators, warps 2..9 drain TMEM (warp w reads
-// lanes 32*(w%4) of half (w-2)/4), add the residual, round and store.
+// CTA: 128 rows x BN (32..256) output columns x one K split. The canvas has
+// only B*C rows and the activation block A is re-read by every column tile, so
+// a 128-row tile keeps the bytes per K block small (16 KB of A + BN*128 B of W)
+// while giving 2 CTAs per column tile for a 256-row canvas. The column tile is
+// chosen so that about one CTA per SM is launched; K is split only when even
+// 32-column tiles leave SMs idle. K-loop of 64-wide blocks through a TMA ring
+// of ~200 KB. Warp 0 issues TMA, warp 1 allocates TMEM and issues the MMAs
+// (M=128, N=BN, K=16), warps 2..5 drain TMEM (warp w reads lanes 32*(w%4)).
+// With one split they add the residual, round and store; with several, every
+// CTA writes its f32 partial and a reduction kernel sums the partials in split
+// order (the result does not depend on which CTA finishes first), adds the
+// residual and stores.
 #include "dg_internal.cuh"
 #include "dg_sm100.cuh"
 #include "dg_tmap.cuh"
@@ -18,20 +25,23 @@ namespace gemmtc {
 
 using namespace sm100;
 
-constexpr int kStages = 5;
 constexpr int kBK = 64;
-constexpr int kBN = 64;
-constexpr int kHalfBytes = 128 * 128;           // 128 rows x 128 B
-constexpr int kABytes = 2 * kHalfBytes;         // 32 KB
-constexpr int kBBytes = kBN * 128;              // 8 KB
-constexpr int kStageBytes = kABytes + kBBytes;  // 40 KB
-constexpr int kThreads = 320;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr int kBM = 128;                        // rows per CTA
+constexpr int kABytes = kBM * 128;              // 16 KB per 64-wide K block
+constexpr int kThreads = 192;                   // TMA warp, MMA warp, 4 epilogue warps
+
+template <int BN> struct Cfg {
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+};
 
 struct Seg {
   __nv_bfloat16* out;  // [M][ldo]
   int ldo;             // row stride of out (elements) = N of this segment
-  int tiles;           // number of 64-column tiles in this segment
+  int tiles;           // number of BN-column tiles in this segment
+  int col0;            // first column of this segment in the split-K partial buffer
 };
 
 struct Params {
@@ -39,35 +49,131 @@ struct Params {
   int nseg;
   Seg seg[3];
   const __nv_bfloat16* R;  // residual [M][ldo of segment 0] or null (single-segment use)
+  int splits;              // K splits (gridDim.z)
+  int ncols;               // total columns over the segments (partial buffer row length)
+  float* part;             // [splits][M][ncols] f32 (splits > 1)
   int* err;
 };
+
+// Sum of the K-split partials in split order, plus the residual, rounded to
+// bf16 and scattered to the output segments. 8 columns per thread; every
+// split's loads are issued before the sum.
+struct ReduceParams {
+  const float* part;
+  int splits, M, ncols;
+  int nseg;
+  __nv_bfloat16* out[3];
+  int col0[4];  // segment column starts (col0[nseg] = ncols)
+  const __nv_bfloat16* R;
+};
+
+template <int MAXS>
+__global__ void __launch_bounds__(256) gemm_reduce_kernel(ReduceParams p) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // 8-column group
+  const int groups = p.ncols / 8;
+  if (idx >= (long long)p.M * groups) return;
+  const int row = (int)(idx / groups);
+  const int col = (int)(idx % groups) * 8;
+  float4 a[MAXS][2];
+#pragma unroll
+  for (int z = 0; z < MAXS; ++z) {
+    if (z < p.splits) {
+      const float4* src = reinterpret_cast<const float4*>(p.part + ((size_t)z * p.M + row) * p.ncols + col);
+      a[z][0] = __ldcg(src);
+      a[z][1] = __ldcg(src + 1);
+    }
+  }
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int z = 0; z < MAXS; ++z) {
+    if (z < p.splits) {
+      acc[0] += a[z][0].x; acc[1] += a[z][0].y; acc[2] += a[z][0].z; acc[3] += a[z][0].w;
+      acc[4] += a[z][1].x; acc[5] += a[z][1].y; acc[6] += a[z][1].z; acc[7] += a[z][1].w;
+    }
+  }
+  int seg = 0;
+  while (seg + 1 < p.nseg && col >= p.col0[seg + 1]) ++seg;
+  const int ldo = p.col0[seg + 1] - p.col0[seg];
+  const size_t o = (size_t)row * ldo + (col - p.col0[seg]);
+  if (p.R) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p.R + o);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(b2[j]);
+      acc[2 * j] += f.x;
+      acc[2 * j + 1] += f.y;
+    }
+  }
+  uint4 w;
+  __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) w2[j] = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+  *reinterpret_cast<uint4*>(p.out[seg] + o) = w;
+}
 
 struct Maps {
   CUtensorMap a;
   CUtensorMap b[3];
 };
 
+// Rounds 32 f32 values to bf16 (+ residual) and stores them at dst.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const __nv_bfloat16* res, const float* v) {
+  float w[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) w[i] = v[i];
+  if (res) {
+    const uint4* rs = reinterpret_cast<const uint4*>(res);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint4 u = rs[c];
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(b2[j]);
+        w[c * 8 + 2 * j] += f.x;
+        w[c * 8 + 2 * j + 1] += f.y;
+      }
+    }
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 u;
+    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b2[j] = __floats2bfloat162_rn(w[c * 8 + 2 * j], w[c * 8 + 2 * j + 1]);
+    d4[c] = u;
+  }
+}
+
+// CTA (column tile, 128-row block, K split). With one split the epilogue adds
+// the residual, rounds to bf16 and stores; with several it writes the f32
+// partial of its K range for gemm_reduce_kernel.
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ Maps maps, Params p) {
+  using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * 256;
-  const int halves = (p.M - m0 > 128) ? 2 : 1;
-  // output segment of this column tile
+  const int m0 = blockIdx.y * kBM;
   int seg = 0, t = blockIdx.x;
   while (seg + 1 < p.nseg && t >= p.seg[seg].tiles) t -= p.seg[seg++].tiles;
-  const int n0 = t * kBN;
+  const int n0 = t * BN;
   const CUtensorMap* mapB = &maps.b[seg];
-  const int nk = p.K / kBK;
+  const int nk_all = p.K / kBK;
+  const int z = blockIdx.z;
+  const int kb0 = (int)(((long long)z * nk_all) / p.splits);
+  const int kb1 = (int)(((long long)(z + 1) * nk_all) / p.splits);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -76,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 128);
+    tmem_alloc(tmem_holder, BN < 32 ? 32 : BN);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -92,93 +198,72 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (lane == 0) {
       const uint64_t polA = policy_evict_last();
       const uint64_t polB = policy_evict_first();
-      const uint32_t bytes = halves * kHalfBytes + kBBytes;
+      const uint32_t bytes = kABytes + C::kBBytes;  // A rows past M are zero-filled
       int s = 0;
       uint32_t ph = 0;
-      bool issued[kStages];
-      uint32_t issued_ph[kStages];
-      for (int i = 0; i < kStages; ++i) issued[i] = false, issued_ph[i] = 0;
-      for (int kb = 0; kb < nk; ++kb) {
+      bool issued[C::kStages];
+      uint32_t issued_ph[C::kStages];
+      for (int i = 0; i < C::kStages; ++i) issued[i] = false, issued_ph[i] = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
-        uint8_t* st = smem + s * kStageBytes;
+        uint8_t* st = smem + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full[s], bytes);
-        for (int h = 0; h < halves; ++h) tma_load_2d(st + h * kHalfBytes, &maps.a, &full[s], kb * kBK, m0 + h * 128, polA);
+        tma_load_2d(st, &maps.a, &full[s], kb * kBK, m0, polA);
         tma_load_2d(st + kABytes, mapB, &full[s], kb * kBK, n0, polB);
         issued[s] = true;
         issued_ph[s] = ph;
-        if (++s == kStages) { s = 0; ph ^= 1u; }
+        if (++s == C::kStages) { s = 0; ph ^= 1u; }
       }
       if (*abort_flag)
-        for (int i = 0; i < kStages; ++i)
+        for (int i = 0; i < C::kStages; ++i)
           if (issued[i]) mbar_wait(&full[i], issued_ph[i], p.err, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, kBN);
+      const uint32_t idesc = idesc_bf16_f32(128, BN);
       int s = 0;
       uint32_t ph = 0;
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full[s], ph, p.err, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(smem + s * kStageBytes);
+        const uint32_t a0 = smem_u32(smem + s * C::kStageBytes);
         const uint32_t b0 = a0 + kABytes;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h < halves) {
-#pragma unroll
-            for (int k = 0; k < kBK / 16; ++k)
-              mma_bf16_ss(tmem + h * kBN, umma_desc_sw128(a0 + h * kHalfBytes + k * 32, 16, 1024),
-                          umma_desc_sw128(b0 + k * 32, 16, 1024), idesc, (kb | k) != 0);
-          }
-        }
+        for (int k = 0; k < kBK / 16; ++k)
+          mma_bf16_ss(tmem, umma_desc_sw128(a0 + k * 32, 16, 1024), umma_desc_sw128(b0 + k * 32, 16, 1024), idesc,
+                      (kb > kb0 || k != 0) ? 1u : 0u);
         mma_commit(&empty[s]);
-        if (++s == kStages) { s = 0; ph ^= 1u; }
+        if (++s == C::kStages) { s = 0; ph ^= 1u; }
       }
       mma_commit(tfull);  // also covers every MMA above before TMEM is read or freed
     }
-  } else {
-    const int ew = warp - 2;
-    const int half = ew >> 2;
+  }
+  // ---------------------------------------------------------------- epilogue
+  if (warp >= 2) {
     const int quad = warp & 3;
-    const int row = m0 + half * 128 + quad * 32 + lane;
+    const int row = m0 + quad * 32 + lane;
+    const Seg sg = p.seg[seg];
     const bool ok = mbar_wait(tfull, 0, p.err, abort_flag);
     tc_fence_after();
-    if (ok && half < halves) {
-      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * kBN);
-      uint32_t r0[32], r1[32];
-      tmem_ld32_sync(tbase, r0);
-      tmem_ld32_sync(tbase + 32, r1);
-      if (row < p.M) {
-        const Seg sg = p.seg[seg];
-        __nv_bfloat16* dst = sg.out + (size_t)row * sg.ldo + n0;
-        float v[64];
+    if (ok) {
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {  // 32 columns at a time
+        float v[32];
+        uint32_t r[32];
+        tmem_ld32_sync(tbase + c * 32, r);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          v[i] = __uint_as_float(r0[i]);
-          v[32 + i] = __uint_as_float(r1[i]);
-        }
-        if (p.R) {
-          const uint4* rs = reinterpret_cast<const uint4*>(p.R + (size_t)row * sg.ldo + n0);
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+        if (row < p.M) {
+          if (p.splits == 1) {
+            store_row32(sg.out + (size_t)row * sg.ldo + n0 + c * 32,
+                        p.R ? p.R + (size_t)row * sg.ldo + n0 + c * 32 : nullptr, v);
+          } else {  // this split's f32 partial; gemm_reduce_kernel sums the splits in order
+            float4* dst =
+                reinterpret_cast<float4*>(p.part + ((size_t)z * p.M + row) * p.ncols + sg.col0 + n0 + c * 32);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 u = rs[c];
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float2 f = __bfloat1622float2(b2[j]);
-              v[c * 8 + 2 * j] += f.x;
-              v[c * 8 + 2 * j + 1] += f.y;
-            }
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
-        }
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 u;
-          __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) b2[j] = __floats2bfloat162_rn(v[c * 8 + 2 * j], v[c * 8 + 2 * j + 1]);
-          d4[c] = u;
         }
       }
     }
@@ -187,17 +272,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, BN < 32 ? 32 : BN);
   }
 }
 
 }  // namespace gemmtc
 
 // ---------------------------------------------------------------- host side
-bool gemm_tc_prepare(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W, void* const* out,
-                     const int* N) {
-  if (cudaFuncSetAttribute(gemmtc::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           gemmtc::kSmemBytes) != cudaSuccess) {
+constexpr int kMaxSplits = 16;
+
+bool gemm_tc_prepare_with(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W,
+                          void* const* out, const int* N, int bn, int splits) {
+  if (cudaFuncSetAttribute(gemmtc::gemm_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gemmtc::Cfg<32>::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(gemmtc::gemm_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gemmtc::Cfg<64>::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(gemmtc::gemm_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gemmtc::Cfg<128>::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(gemmtc::gemm_tc_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           gemmtc::Cfg<256>::kSmemBytes) != cudaSuccess) {
     set_last_error("cudaFuncSetAttribute(gemm_tc_kernel) failed");
     return false;
   }
@@ -207,45 +300,124 @@ bool gemm_tc_prepare(GemmTc* g, const void* A, int M, int K, int nseg, const voi
   }
   static_assert(sizeof(gemmtc::Maps) <= sizeof(g->maps), "GemmTc map storage too small");
   gemmtc::Maps* maps = reinterpret_cast<gemmtc::Maps*>(g->maps);
+  int ncols = 0, gcd = 256;
+  for (int i = 0; i < nseg; ++i) {
+    if (N[i] % 32 != 0) {
+      set_last_error("gemm_tc: N must be a multiple of 32");
+      return false;
+    }
+    while (N[i] % gcd) gcd >>= 1;
+    ncols += N[i];
+  }
+  if (bn != 32 && bn != 64 && bn != 128 && bn != 256) bn = 64;
+  if (gcd < bn) {
+    set_last_error("gemm_tc: column tile wider than a segment allows");
+    return false;
+  }
+  g->bn = bn;
   const uint64_t dA[2] = {(uint64_t)K, (uint64_t)M};
   const uint64_t sA[1] = {(uint64_t)K * 2};
-  const uint32_t bA[2] = {64, 128};
+  const uint32_t bA[2] = {64, (uint32_t)gemmtc::kBM};
   if (!encode_tmap_bf16(&maps->a, A, 2, dA, sA, bA, true)) return false;
   g->M = M;
   g->K = K;
   g->nseg = nseg;
   g->tiles = 0;
+  g->ncols = ncols;
   for (int i = 0; i < nseg; ++i) {
-    if (N[i] % gemmtc::kBN != 0) {
-      set_last_error("gemm_tc: N must be a multiple of 64");
-      return false;
-    }
     const uint64_t dB[2] = {(uint64_t)K, (uint64_t)N[i]};
-    const uint32_t bB[2] = {64, (uint32_t)gemmtc::kBN};
+    const uint32_t bB[2] = {64, (uint32_t)g->bn};
     if (!encode_tmap_bf16(&maps->b[i], W[i], 2, dB, sA, bB, true)) return false;
     g->out[i] = out[i];
     g->N[i] = N[i];
-    g->tiles += N[i] / gemmtc::kBN;
+    g->tiles += N[i] / g->bn;
   }
+  g->splits = std::max(1, std::min(std::min(splits, kMaxSplits), K / 64));
   return true;
 }
+
+bool gemm_tc_prepare(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W, void* const* out,
+                     const int* N, int sm_count) {
+  int gcd = 256;
+  for (int i = 0; i < nseg; ++i)
+    while (gcd > 32 && N[i] % gcd) gcd >>= 1;
+  // Column tile by a cost model: waves of CTAs x bytes each CTA moves per K
+  // block (16 KB of A + bn * 128 B of W); ties go to the wider tile. K is
+  // split only when the best choice still leaves most SMs idle.
+  const int mblocks = ceil_div(M, gemmtc::kBM);
+  auto ctas = [&](int w) {
+    int tiles = 0;
+    for (int i = 0; i < nseg; ++i) tiles += N[i] / w;
+    return tiles * mblocks;
+  };
+  int bn = gcd;
+  long long best = -1;
+  for (int w = gcd; w >= 32; w >>= 1) {
+    const long long cost = (long long)ceil_div(ctas(w), sm_count) * (gemmtc::kABytes + w * 128);
+    if (best < 0 || cost < best) {
+      best = cost;
+      bn = w;
+    }
+  }
+  int splits = 1;
+  if (ctas(bn) * 2 <= sm_count) splits = std::max(1, std::min(sm_count / ctas(bn), (K / 64) / 4));
+  return gemm_tc_prepare_with(g, A, M, K, nseg, W, out, N, bn, splits);
+}
+
+size_t gemm_tc_partial_floats(const GemmTc& g) {
+  return g.splits > 1 ? (size_t)g.splits * g.M * g.ncols : 0;
+}
+size_t gemm_tc_counters(const GemmTc&) { return 0; }
 
 void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual) {
   gemmtc::Params p;
   p.M = g.M;
   p.K = g.K;
   p.nseg = g.nseg;
+  int col0 = 0;
   for (int i = 0; i < 3; ++i) {
     p.seg[i].out = i < g.nseg ? static_cast<__nv_bfloat16*>(g.out[i]) : nullptr;
     p.seg[i].ldo = i < g.nseg ? g.N[i] : 0;
-    p.seg[i].tiles = i < g.nseg ? g.N[i] / gemmtc::kBN : 0;
+    p.seg[i].tiles = i < g.nseg ? g.N[i] / g.bn : 0;
+    p.seg[i].col0 = col0;
+    if (i < g.nseg) col0 += g.N[i];
   }
   p.R = static_cast<const __nv_bfloat16*>(residual);
+  p.splits = g.splits;
+  p.ncols = g.ncols;
+  p.part = g.part;
   p.err = ex.err;
-  dim3 grid(g.tiles, ceil_div(g.M, 256));
-  gemmtc::gemm_tc_kernel<<<grid, gemmtc::kThreads, gemmtc::kSmemBytes, ex.stream>>>(
-      *reinterpret_cast<const gemmtc::Maps*>(g.maps), p);
+  dim3 grid(g.tiles, ceil_div(g.M, gemmtc::kBM), g.splits);
+  const gemmtc::Maps& maps = *reinterpret_cast<const gemmtc::Maps*>(g.maps);
+  if (g.bn == 32)
+    gemmtc::gemm_tc_kernel<32><<<grid, gemmtc::kThreads, gemmtc::Cfg<32>::kSmemBytes, ex.stream>>>(maps, p);
+  else if (g.bn == 256)
+    gemmtc::gemm_tc_kernel<256><<<grid, gemmtc::kThreads, gemmtc::Cfg<256>::kSmemBytes, ex.stream>>>(maps, p);
+  else if (g.bn == 128)
+    gemmtc::gemm_tc_kernel<128><<<grid, gemmtc::kThreads, gemmtc::Cfg<128>::kSmemBytes, ex.stream>>>(maps, p);
+  else
+    gemmtc::gemm_tc_kernel<64><<<grid, gemmtc::kThreads, gemmtc::Cfg<64>::kSmemBytes, ex.stream>>>(maps, p);
   ex.launches++;
+  if (g.splits > 1) {
+    gemmtc::ReduceParams r;
+    r.part = g.part;
+    r.splits = g.splits;
+    r.M = g.M;
+    r.ncols = g.ncols;
+    r.nseg = g.nseg;
+    int c = 0;
+    for (int i = 0; i < 3; ++i) {
+      r.out[i] = i < g.nseg ? static_cast<__nv_bfloat16*>(g.out[i]) : nullptr;
+      r.col0[i] = c;
+      if (i < g.nseg) c += g.N[i];
+    }
+    r.col0[3] = c;
+    for (int i = g.nseg; i < 3; ++i) r.col0[i + 1] = c;
+    r.R = static_cast<const __nv_bfloat16*>(residual);
+    const long long threads = (long long)g.M * (g.ncols / 8);
+    gemmtc::gemm_reduce_kernel<kMaxSplits><<<(unsigned)ceil_div((int)threads, 256), 256, 0, ex.stream>>>(r);
+    ex.launches++;
+  }
 }
 
 }  // namespace dg

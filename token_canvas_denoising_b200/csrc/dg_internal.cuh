@@ -69,12 +69,21 @@ void launch_lmhead_tc(Exec& ex, const CUtensorMap& tmA, const CUtensorMap& tmB, 
 // segments sharing A; prepared once (tensor maps), launched many times.
 struct alignas(64) GemmTc {
   unsigned char maps[4 * 128];  // CUtensorMap for A and each W_i
-  int M = 0, K = 0, nseg = 0, tiles = 0;
+  int M = 0, K = 0, nseg = 0, tiles = 0, bn = 64, splits = 1, ncols = 0;
   void* out[3] = {nullptr, nullptr, nullptr};
   int N[3] = {0, 0, 0};
+  float* part = nullptr;         // split-K partials [splits][M][ncols]
+  unsigned* counters = nullptr;  // per output tile, zero between launches
 };
+// Chooses the tile width and the K splits (for sm_count SMs) and encodes the
+// tensor maps; the caller then provides `part` and zeroed `counters` of the
+// sizes below when splits > 1.
 bool gemm_tc_prepare(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W, void* const* out,
-                     const int* N);
+                     const int* N, int sm_count);
+bool gemm_tc_prepare_with(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W,
+                          void* const* out, const int* N, int bn, int splits);
+size_t gemm_tc_partial_floats(const GemmTc& g);
+size_t gemm_tc_counters(const GemmTc& g);
 void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual);
 
 // tcgen05 attention (bf16, head_dim 128): tensor maps per group of up to 8

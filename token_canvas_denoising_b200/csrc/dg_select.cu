@@ -57,12 +57,21 @@ __device__ __forceinline__ EntStats load_rec(const LmRec* r) {
   return {a.x, a.y, a.z, a.w, b.x};
 }
 
+// Orderable 32-bit image of a float (total order, negatives below positives).
+__device__ __forceinline__ uint32_t float_order(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kMaxRecPerLane = 8;  // partials preloaded per lane (P <= 256 in one pass)
+
 // Grid (ceil(C/8), B), 256 threads. Phase 1: one warp per canvas row folds the
-// row's P partials (lane j takes partials j, j+32, ...; then a fixed xor
-// butterfly), giving ent = ln Z - S/Z and the argmax. Phase 2 runs in the last
-// block of each canvas to arrive: rank-by-count selection of the k smallest
-// (entropy, position) keys among unfrozen positions, freeze, stop test,
-// re-noise. The last canvas to finish sets the all-done flag.
+// row's P partials (lane j takes partials j, j+32, ..., all loaded before the
+// fold; then a fixed xor butterfly), giving ent = ln Z - S/Z and the argmax.
+// Phase 2 runs in the last block of each canvas to arrive: each unfrozen
+// position counts the unfrozen positions with a smaller (entropy, position)
+// key; the k with rank < k freeze to their argmax; stop test; re-noise. The
+// last canvas to finish sets the all-done flag.
 __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -71,7 +80,16 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
     const int r = b * a.C + p_row;
     const LmRec* rec = a.part.rec + (size_t)r * a.part.P;
     EntStats st = ent_empty();
-    for (int j = lane; j < a.part.P; j += 32) st = ent_merge(st, load_rec(rec + j));
+    for (int j0 = 0; j0 < a.part.P; j0 += 32 * kMaxRecPerLane) {
+      EntStats buf[kMaxRecPerLane];
+#pragma unroll
+      for (int u = 0; u < kMaxRecPerLane; ++u) {
+        const int j = j0 + lane + 32 * u;
+        buf[u] = (j < a.part.P) ? load_rec(rec + j) : ent_empty();
+      }
+#pragma unroll
+      for (int u = 0; u < kMaxRecPerLane; ++u) st = ent_merge(st, buf[u]);
+    }
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       EntStats ot;
@@ -102,8 +120,7 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
   if (!s_last) return;
   __threadfence();
 
-  __shared__ float s_ent[256];
-  __shared__ uint8_t s_unf[256];
+  __shared__ __align__(16) unsigned long long s_key[256];
   __shared__ float s_min[8];
   const int p = threadIdx.x;
   const bool valid = p < a.C;
@@ -115,8 +132,10 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
     float e = valid ? __ldcg(&a.ent[r]) : INFINITY;
     if (!(e == e)) e = INFINITY;  // NaN (already flagged) orders last
     const bool unf = valid && a.frozen[r] == 0;
-    s_ent[p] = e;
-    s_unf[p] = unf ? 1 : 0;
+    // key = (entropy, position); frozen and padding slots sort after every unfrozen one
+    const unsigned long long key =
+        unf ? (((unsigned long long)float_order(e) << 32) | (unsigned)p) : ~0ull;
+    s_key[p] = key;
     const int U = __syncthreads_count(unf);
     const int t = a.step[b];
     const int left = a.max_steps - t;
@@ -124,9 +143,11 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
     bool F = false;
     if (unf) {
       int rank = 0;
-      for (int q = 0; q < a.C; ++q) {
-        const float eq = s_ent[q];
-        rank += (s_unf[q] && (eq < e || (eq == e && q < p))) ? 1 : 0;
+      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(s_key);
+#pragma unroll 8
+      for (int q = 0; q < 128; ++q) {
+        const ulonglong2 kq = k2[q];
+        rank += (kq.x < key) + (kq.y < key);
       }
       F = rank < k;
     }
@@ -153,7 +174,6 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
       a.tok[r] = canvas_draw(a.seed[b], (uint32_t)(t + 1), (uint32_t)p, (uint32_t)b, (uint32_t)a.V);
     }
     if (valid && a.fmask) a.fmask[r] = F ? 1 : 0;
-    __syncthreads();
     if (threadIdx.x == 0) {
       a.step[b] = t + 1;
       if (stop) a.done[b] = 1;

@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
+  griddep_launch();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -134,11 +135,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool issued_q = false;
       bool issued[2] = {false, false};
       uint32_t iph[2] = {0, 0};
+      // the prompt prefix is an input of the step: its first tiles may be
+      // fetched before the predecessor kernels are done
+      int pre = 0;
+      while (pre < 2 && pre < n && t0 + pre < nps) {
+        const int s = pre;
+        uint8_t* kb = smem + kOffKV + s * 2 * kMatBytes;
+        mbar_arrive_expect_tx(&k_full[s], kMatBytes);
+        for (int a = 0; a < 2; ++a) tma_load_2d(kb + a * kAtom, &maps.pk[lb], &k_full[s], g * 128 + a * 64, (t0 + pre) * kTile, pol);
+        mbar_arrive_expect_tx(&v_full[s], kMatBytes);
+        for (int a = 0; a < 2; ++a)
+          tma_load_2d(kb + kMatBytes + a * kAtom, &maps.pv[lb], &v_full[s], g * 128 + a * 64, (t0 + pre) * kTile, pol);
+        issued[s] = true;
+        iph[s] = 0;
+        ++pre;
+      }
+      griddep_wait();
       mbar_arrive_expect_tx(q_full, kMatBytes);
       for (int a = 0; a < 2; ++a)
         tma_load_2d(smem + kOffQ + a * kAtom, &maps.q, q_full, qh * 128 + a * 64, b * p.C + qt * kTile, pol);
       issued_q = true;
-      for (int i = 0; i < n && !*abort_flag; ++i) {
+      for (int i = pre; i < n && !*abort_flag; ++i) {
         const int s = i & 1;
         if (i >= 2 && !mbar_wait(&kv_empty[s], ((i >> 1) - 1) & 1, p.err, abort_flag)) break;
         const int j = t0 + i;
@@ -174,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    griddep_wait();
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(128, 128, false);
       const uint32_t id_pv = idesc_bf16_f32(128, 128, true);
@@ -210,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ softmax
+    griddep_wait();
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // query row within the tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -333,6 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 // O = sum_z w_z O_z / sum_z w_z l_z. One warp per (row, head), 4 dims per lane.
 __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                   __nv_bfloat16* __restrict__ O, int rows_total, int splits) {
+  griddep_launch();
+  griddep_wait();
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= rows_total) return;
@@ -435,13 +456,14 @@ void launch_attn_tc(Exec& ex, const AttnTc& at) {
     p.part_ml = at.part_ml;
     p.err = ex.err;
     dim3 grid(q_tiles * sh.Hq, grp.nreq, at.splits);
-    attntc::attn_tc_kernel<<<grid, attntc::kThreads, attntc::kSmemBytes, ex.stream>>>(
-        *reinterpret_cast<const attntc::Maps*>(grp.maps), p);
+    launch_pdl(attntc::attn_tc_kernel, grid, dim3(attntc::kThreads), attntc::kSmemBytes, ex.stream,
+               *reinterpret_cast<const attntc::Maps*>(grp.maps), p);
     ex.launches++;
   }
   if (at.splits > 1) {
-    attntc::attn_merge_kernel<<<ceil_div(rows_total, 8), 256, 0, ex.stream>>>(
-        at.part_o, at.part_ml, static_cast<__nv_bfloat16*>(at.O), rows_total, at.splits);
+    launch_pdl(attntc::attn_merge_kernel, dim3(ceil_div(rows_total, 8)), dim3(256), 0, ex.stream,
+               (const float*)at.part_o, (const float*)at.part_ml, static_cast<__nv_bfloat16*>(at.O), rows_total,
+               at.splits);
     ex.launches++;
   }
 }

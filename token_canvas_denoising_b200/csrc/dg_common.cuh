@@ -78,6 +78,15 @@ __host__ __device__ __forceinline__ int32_t canvas_draw(uint64_t seed, uint32_t 
   return (int32_t)(((o.x0 >> 32) * (uint64_t)vocab) >> 32);
 }
 
+// ---------------------------------------------------------------- launch order
+// Programmatic dependent launch: a kernel may start while its predecessor in
+// the stream is still running. Each kernel calls griddep_launch() early (its
+// dependents may then be scheduled) and griddep_wait() before it touches any
+// memory a predecessor writes (or reads); work before the wait is limited to
+// set-up and loads of read-only weights.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- misc
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 

@@ -69,6 +69,8 @@ struct ReduceParams {
 
 template <int MAXS>
 __global__ void __launch_bounds__(256) gemm_reduce_kernel(ReduceParams p) {
+  griddep_launch();
+  griddep_wait();
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // 8-column group
   const int groups = p.ncols / 8;
   if (idx >= (long long)p.M * groups) return;
@@ -185,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     tmem_alloc(tmem_holder, BN < 32 ? 32 : BN);
     tmem_relinquish();
   }
+  griddep_launch();
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&maps.a);
     tma_prefetch_desc(mapB);
@@ -204,7 +207,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       bool issued[C::kStages];
       uint32_t issued_ph[C::kStages];
       for (int i = 0; i < C::kStages; ++i) issued[i] = false, issued_ph[i] = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      // weights are read-only inputs: the first stages' W tiles are fetched
+      // before waiting for the kernel that produces A
+      const int pre = min(C::kStages, kb1 - kb0);
+      for (int i = 0; i < pre; ++i) {
+        uint8_t* st = smem + i * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[i], bytes);
+        tma_load_2d(st + kABytes, mapB, &full[i], (kb0 + i) * kBK, n0, polB);
+        issued[i] = true;
+        issued_ph[i] = 0;
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * C::kStageBytes, &maps.a, &full[i], (kb0 + i) * kBK, m0, polA);
+      s = pre % C::kStages;
+      ph = (pre == C::kStages) ? 1u : 0u;
+      for (int kb = kb0 + pre; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
         uint8_t* st = smem + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full[s], bytes);
@@ -240,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   }
   // ---------------------------------------------------------------- epilogue
   if (warp >= 2) {
+    griddep_wait();  // the residual and the outputs belong to earlier kernels
     const int quad = warp & 3;
     const int row = m0 + quad * 32 + lane;
     const Seg sg = p.seg[seg];
@@ -389,14 +407,15 @@ void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual) {
   p.err = ex.err;
   dim3 grid(g.tiles, ceil_div(g.M, gemmtc::kBM), g.splits);
   const gemmtc::Maps& maps = *reinterpret_cast<const gemmtc::Maps*>(g.maps);
+  const dim3 block(gemmtc::kThreads);
   if (g.bn == 32)
-    gemmtc::gemm_tc_kernel<32><<<grid, gemmtc::kThreads, gemmtc::Cfg<32>::kSmemBytes, ex.stream>>>(maps, p);
+    launch_pdl(gemmtc::gemm_tc_kernel<32>, grid, block, gemmtc::Cfg<32>::kSmemBytes, ex.stream, maps, p);
   else if (g.bn == 256)
-    gemmtc::gemm_tc_kernel<256><<<grid, gemmtc::kThreads, gemmtc::Cfg<256>::kSmemBytes, ex.stream>>>(maps, p);
+    launch_pdl(gemmtc::gemm_tc_kernel<256>, grid, block, gemmtc::Cfg<256>::kSmemBytes, ex.stream, maps, p);
   else if (g.bn == 128)
-    gemmtc::gemm_tc_kernel<128><<<grid, gemmtc::kThreads, gemmtc::Cfg<128>::kSmemBytes, ex.stream>>>(maps, p);
+    launch_pdl(gemmtc::gemm_tc_kernel<128>, grid, block, gemmtc::Cfg<128>::kSmemBytes, ex.stream, maps, p);
   else
-    gemmtc::gemm_tc_kernel<64><<<grid, gemmtc::kThreads, gemmtc::Cfg<64>::kSmemBytes, ex.stream>>>(maps, p);
+    launch_pdl(gemmtc::gemm_tc_kernel<64>, grid, block, gemmtc::Cfg<64>::kSmemBytes, ex.stream, maps, p);
   ex.launches++;
   if (g.splits > 1) {
     gemmtc::ReduceParams r;
@@ -415,7 +434,8 @@ void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual) {
     for (int i = g.nseg; i < 3; ++i) r.col0[i + 1] = c;
     r.R = static_cast<const __nv_bfloat16*>(residual);
     const long long threads = (long long)g.M * (g.ncols / 8);
-    gemmtc::gemm_reduce_kernel<kMaxSplits><<<(unsigned)ceil_div((int)threads, 256), 256, 0, ex.stream>>>(r);
+    launch_pdl(gemmtc::gemm_reduce_kernel<kMaxSplits>, dim3((unsigned)ceil_div((int)threads, 256)), dim3(256), 0,
+               ex.stream, r);
     ex.launches++;
   }
 }

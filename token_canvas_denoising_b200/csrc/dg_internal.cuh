@@ -4,6 +4,7 @@
 #include <cuda.h>
 
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "dg_canvas.h"
@@ -48,6 +49,25 @@ struct AttnShape {
 };
 
 void set_last_error(const std::string& msg);
+
+// Launch with programmatic stream serialization (see griddep_wait in
+// dg_common.cuh); the kernel must call griddep_wait() before using its
+// predecessors' outputs.
+template <typename... KArgs, typename... Args>
+inline void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---- embed / linear / attention / LM head (dtype-dispatched)
 void launch_embed(Exec& ex, int dtype, const void* E, const int32_t* tok, void* X, int M, int d, int V);

@@ -94,6 +94,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
+  griddep_launch();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -109,11 +110,33 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t issued_ph[kStages];
       bool issued[kStages];
       for (int i = 0; i < kStages; ++i) issued[i] = false, issued_ph[i] = 0;
+      // vocab weights are read-only inputs: the first stages' W tiles are
+      // fetched before waiting for the kernel that produces Hs
+      int pre = 0;
+      if (n_tiles > 0) {
+        const int ng0 = min(kMaxGran, g1 - g0);
+        const uint32_t bytes0 = halves * kHalfBytes + ng0 * kGranBytes;
+        pre = min(kStages, nk);
+        for (int i = 0; i < pre; ++i) {
+          uint8_t* st = smem + i * kStageBytes;
+          mbar_arrive_expect_tx(&full[i], bytes0);
+          for (int g = 0; g < ng0; ++g)
+            tma_load_2d(st + kABytes + g * kGranBytes, &tmB, &full[i], i * kBK, (g0 + g) * kGranule, polB);
+          issued[i] = true;
+          issued_ph[i] = 0;
+        }
+        griddep_wait();
+        for (int i = 0; i < pre; ++i)
+          for (int h = 0; h < halves; ++h)
+            tma_load_2d(smem + i * kStageBytes + h * kHalfBytes, &tmA, &full[i], i * kBK, m0 + h * 128, polA);
+        s = pre % kStages;
+        ph = (pre == kStages) ? 1u : 0u;
+      }
       for (int t = 0; t < n_tiles && !*abort_flag; ++t) {
         const int gt = g0 + t * kMaxGran;
         const int ng = min(kMaxGran, g1 - gt);
         const uint32_t bytes = halves * kHalfBytes + ng * kGranBytes;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = (t == 0 ? pre : 0); kb < nk; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
           uint8_t* st = smem + s * kStageBytes;
           mbar_arrive_expect_tx(&full[s], bytes);
@@ -172,6 +195,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   } else {
     // ---------------------------------------------------------------- epilogue
+    griddep_wait();  // invT and the partial records belong to earlier kernels
     const int ew = warp - 2;
     const int half = ew >> 2;
     const int quad = warp & 3;
@@ -287,7 +311,7 @@ void launch_lmhead_tc(Exec& ex, const CUtensorMap& tmA, const CUtensorMap& tmB, 
   p.rec = part.rec;
   p.err = ex.err;
   dim3 grid(part.P, ceil_div(M, 256));
-  lmtc::lmhead_tc_kernel<<<grid, lmtc::kThreads, lmtc::kSmemBytes, ex.stream>>>(tmA, tmB, p);
+  launch_pdl(lmtc::lmhead_tc_kernel, grid, dim3(lmtc::kThreads), lmtc::kSmemBytes, ex.stream, tmA, tmB, p);
   ex.launches++;
 }
 

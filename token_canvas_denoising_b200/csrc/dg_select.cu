@@ -73,6 +73,8 @@ constexpr int kMaxRecPerLane = 8;  // partials preloaded per lane (P <= 256 in o
 // key; the k with rank < k freeze to their argmax; stop test; re-noise. The
 // last canvas to finish sets the all-done flag.
 __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
+  griddep_launch();
+  griddep_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p_row = blockIdx.x * 8 + warp;
@@ -219,7 +221,7 @@ void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uin
     a.stop_entropy = sched->stop_entropy;
   }
   dim3 grid(ceil_div(C, 8), B);
-  merge_select_kernel<<<grid, 256, 0, ex.stream>>>(a);
+  launch_pdl(merge_select_kernel, grid, dim3(256), 0, ex.stream, a);
   ex.launches++;
 }
 

@@ -11,6 +11,8 @@ namespace dg {
 template <typename T>
 __global__ void embed_kernel(const T* __restrict__ E, const int32_t* __restrict__ tok,
                              T* __restrict__ X, int d, int V, int* err) {
+  griddep_launch();
+  griddep_wait();
   const int r = blockIdx.x;
   int t = tok[r];
   if (t < 0 || t >= V) {
@@ -27,8 +29,8 @@ void launch_embed(Exec& ex, int dtype, const void* E, const int32_t* tok, void* 
   if (dtype == DG_F32)
     embed_kernel<float><<<M, 128, 0, ex.stream>>>((const float*)E, tok, (float*)X, d, V, ex.err);
   else
-    embed_kernel<__nv_bfloat16><<<M, 128, 0, ex.stream>>>((const __nv_bfloat16*)E, tok, (__nv_bfloat16*)X, d,
-                                                          V, ex.err);
+    launch_pdl(embed_kernel<__nv_bfloat16>, dim3(M), dim3(128), 0, ex.stream, (const __nv_bfloat16*)E, tok,
+               (__nv_bfloat16*)X, d, V, ex.err);
   ex.launches++;
 }
 

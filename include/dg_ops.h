@@ -15,6 +15,7 @@
 #ifndef DG_OPS_H
 #define DG_OPS_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #include "dg_canvas.h"
@@ -32,6 +33,31 @@ extern "C" {
  * bf16 needs d % 64 == 0 and V % 256 == 0; f32 any d % 8 == 0. */
 dg_status dg_lmhead_entropy(int32_t dtype, const void *hs, const void *lm_head, const float *inv_temp,
                             int32_t M, int32_t d, int32_t V, float *ent, int32_t *argmax, void *stream);
+
+/* Allocation-free variant of dg_lmhead_entropy. The pages have no counterpart
+ * to this call: it exists for users of this library who may not allocate
+ * device memory at the point where they run the LM head -- work that is being
+ * recorded into a CUDA graph, or an application whose device memory is
+ * reserved up front by its own allocator.
+ * Same arguments and results as dg_lmhead_entropy. Its temporary per-row
+ * partial results go to a fixed device array inside the library (2 MiB, held
+ * on every GPU that loads the library until the process exits) instead of a
+ * fresh buffer; the call makes no cudaMalloc, cudaFree or other allocation.
+ * Limit: M times the number of vocab partitions (at most the GPU's SM count,
+ * fewer for M > 256) must not exceed dg_lmhead_entropy_noalloc_max_records()
+ * (65,536); larger problems return DG_ERR_UNSUPPORTED.
+ * The first call on each device looks up the array's device address; make
+ * that first call before any stream capture. All calls on a device share the
+ * array: two calls whose work can overlap on the GPU (e.g. on different
+ * streams without ordering between them) race. Nothing in the array needs to
+ * start at zero: each call writes every entry it reads. */
+dg_status dg_lmhead_entropy_noalloc(int32_t dtype, const void *hs, const void *lm_head,
+                                    const float *inv_temp, int32_t M, int32_t d, int32_t V,
+                                    float *ent, int32_t *argmax, void *stream);
+
+/* Capacity of the fixed array used by dg_lmhead_entropy_noalloc, in partial
+ * records (one per row and vocab partition). */
+size_t dg_lmhead_entropy_noalloc_max_records(void);
 
 /* Bidirectional GQA attention of B*C canvas queries over each request's
  * cached prompt K/V followed by the canvas K/V, no mask, scale 1/sqrt(h),

@@ -37,6 +37,24 @@ def lmhead_entropy(hs, lm_head, inv_temp=None):
     return ent, am
 
 
+def lmhead_entropy_noalloc(hs, lm_head, inv_temp=None, ent=None, argmax=None):
+    """Like lmhead_entropy, but the library makes no device allocation: its
+    temporary partial results live in a fixed device array inside the library.
+    Pass preallocated `ent` (f32 [M]) and `argmax` (int32 [M]) to allocate
+    nothing on the Python side either."""
+    lib = L.load()
+    M, d = hs.shape
+    V = lm_head.shape[0]
+    if ent is None:
+        ent = torch.empty(M, dtype=torch.float32, device=hs.device)
+    if argmax is None:
+        argmax = torch.empty(M, dtype=torch.int32, device=hs.device)
+    st = lib.dg_lmhead_entropy_noalloc(_dt(hs), _p(hs), _p(lm_head), _p(inv_temp), M, d, V, _p(ent),
+                                       _p(argmax), _stream())
+    L.check(st, "dg_lmhead_entropy_noalloc")
+    return ent, argmax
+
+
 def attention(q, kc, vc, prefix_k, prefix_v, B, C_len, Hq, Hk, h):
     """Bidirectional GQA attention output [B*C, Hq*h] (see dg_ops.h)."""
     lib = L.load()

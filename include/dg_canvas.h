@@ -106,6 +106,8 @@ typedef struct dg_step_out {
   uint8_t *freeze_mask; /* [B*C] 1 where the position froze at this step        */
   void *attn_out;       /* [B*C][n_q_heads*head_dim] attention output O (dtype) */
   void *hidden;         /* [B*C][d_model] residual stream fed to the LM head   */
+  void *hidden_attn;    /* [B*C][d_model] residual stream after attention and Wo,
+                           before the MoE block (equals `hidden` without MoE)  */
 } dg_step_out;
 
 /* Host-side copy of the decode state (all host arrays). */

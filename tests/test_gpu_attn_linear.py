@@ -55,6 +55,36 @@ def test_attention_matches_oracle(B, C, S, Hq, Hk):
     assert n == 0, f"{n} elements out of tolerance, max abs diff {mx:.3g}"
 
 
+@pytest.mark.parametrize("B,C,S,Hq,Hk,growth", [
+    (1, 128, (1024,), 2, 1, 0.6),    # one work item per head: long walk over growing tiles
+    (4, 256, (2048,) * 4, 16, 8, 0.3),
+])
+def test_attention_growing_scores_rescale(B, C, S, Hq, Hk, growth):
+    """Prefix keys scaled by 1 + growth * (tile index): the scores grow along
+    the sequence, so the running maximum is raised in the middle of the walk,
+    in some query rows of a warp and not in others (the lazy rescale of O)."""
+    from token_canvas_denoising_b200 import ops
+    h = 128
+    seed = 300 + B + C
+    q = fx.normal(seed, 1, (B * C, Hq * h), 1.0, "bf16")
+    kc = fx.normal(seed, 2, (B * C, Hk * h), 1.0, "bf16")
+    vc = fx.normal(seed, 3, (B * C, Hk * h), 1.0, "bf16")
+    pk, pv = [], []
+    for b in range(B):
+        k0 = _bf(fx.normal(seed, 10 + b, (S[b], Hk, h), 1.0, "bf16"))
+        scale = 1.0 + growth * (np.arange(S[b]) // 128)
+        pk.append(fx.f32_to_bf16_bits((k0 * scale[:, None, None]).astype(np.float32)))
+        pv.append(fx.normal(seed, 30 + b, (S[b], Hk, h), 1.0, "bf16"))
+    o = ops.attention(_dev(q), _dev(kc), _dev(vc), [_dev(x) for x in pk], [_dev(x) for x in pv],
+                      B, C, Hq, Hk, h)
+    o = o.float().cpu().numpy().astype(np.float64)
+    model = {"dtype": "bf16", "d": Hq * h, "Hq": Hq, "Hk": Hk, "h": h, "V": 2}
+    ref = om.attention(model, _bf(q).reshape(-1, Hq, h), _bf(kc).reshape(-1, Hk, h),
+                       _bf(vc).reshape(-1, Hk, h), list(zip(pk, pv)), B, C)
+    n, mx = close(o, ref)
+    assert n == 0, f"{n} elements out of tolerance, max abs diff {mx:.3g}"
+
+
 def test_attention_zero_queries_average_values():
     """Q = 0 makes every score 0: each output row is the mean of all S + C value rows."""
     from token_canvas_denoising_b200 import ops

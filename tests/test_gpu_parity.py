@@ -64,6 +64,24 @@ def test_bf16_canvas256_first_steps():
     _run(fx.CONFIGS["canvas256"], n_steps=3, free_running=False)
 
 
+def test_bf16_moe_small_full_decode():
+    """MoE FFN path (router, top-k routing, GeGLU experts, shared expert,
+    combine) on a small model, full decode."""
+    cfg = fx.Config("moe_small", B=1, C=96, S=(150,), d=256, Hq=2, Hk=1, h=128, V=2048, dtype="bf16",
+                    max_steps=8, weight_seed=17, canvas_seeds=(5,), n_experts=32, top_k=4, moe_inter=128,
+                    n_shared=1)
+    _run(cfg)
+
+
+def test_bf16_moe_uneven_experts():
+    """Many experts per token and few tokens: several experts get no token,
+    others several tiles of tokens; I not a multiple of 128."""
+    cfg = fx.Config("moe_uneven", B=2, C=40, S=(64, 0), d=192, Hq=2, Hk=2, h=128, V=1024, dtype="bf16",
+                    max_steps=6, weight_seed=23, canvas_seeds=(1, 2), n_experts=64, top_k=8, moe_inter=192,
+                    n_shared=1)
+    _run(cfg, n_steps=3)
+
+
 def test_decode_block_matches_stepping():
     """dg_decode_block (device loop) ends in the same state as single steps."""
     from token_canvas_denoising_b200.canvas import from_workload, schedule

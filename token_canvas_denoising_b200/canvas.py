@@ -82,8 +82,10 @@ class DenoiseCanvas:
                 "freeze_mask": torch.empty(self.M, dtype=torch.uint8, device=dev),
                 "attn_out": torch.empty(self.M, self._model.n_q_heads * self._model.head_dim, dtype=sdt, device=dev),
                 "hidden": torch.empty(self.M, self._model.d_model, dtype=sdt, device=dev),
+                "hidden_attn": torch.empty(self.M, self._model.d_model, dtype=sdt, device=dev),
             }
-            dbg = L.dg_step_out(*[_ptr(out[k]) for k in ("ent", "argmax", "freeze_mask", "attn_out", "hidden")])
+            dbg = L.dg_step_out(*[_ptr(out[k]) for k in ("ent", "argmax", "freeze_mask", "attn_out", "hidden",
+                                                          "hidden_attn")])
         st = self._lib.dg_denoise_step(self._ctx, C.byref(sched), C.byref(dbg) if dbg is not None else None)
         L.check(st, "dg_denoise_step")
         return out

@@ -82,6 +82,10 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   c->lm.rec = w.take<dg::LmRec>(M * (size_t)c->lm.P);
   c->ent = w.take<float>(M);
   c->am = w.take<int32_t>(M);
+  if (c->m.n_experts) {
+    dg::MoeShape ms{c->M, c->m.d_model, c->m.n_experts, c->m.top_k, c->m.n_shared, c->m.moe_inter};
+    c->moe_ws = w.take<char>(dg::moe_workspace_bytes(ms));
+  }
   if (c->m.dtype == DG_BF16) {
     c->g_qkv.part = w.take<float>(dg::gemm_tc_partial_floats(c->g_qkv));
     c->g_qkv.counters = w.take<unsigned>(dg::gemm_tc_counters(c->g_qkv));
@@ -119,7 +123,10 @@ dg_status validate_model(const dg_model_desc* m) {
                m->n_shared >= 0,
            "MoE sizes");
     DG_ARG(m->w_router && m->w_gate && m->w_up && m->w_down, "an MoE weight pointer is NULL");
-    DG_UNSUP(false, "MoE FFN is not available in this build");
+    DG_UNSUP(m->dtype == DG_BF16, "the MoE FFN needs the bf16 storage dtype");
+    DG_UNSUP(m->n_experts <= 256 && m->n_experts % 32 == 0 && m->top_k <= 8 && m->n_shared <= 2 &&
+                 m->moe_inter % 64 == 0,
+             "MoE needs n_experts <= 256 and a multiple of 32, top_k <= 8, n_shared <= 2, moe_inter % 64 == 0");
   }
   return DG_OK;
 }
@@ -166,6 +173,10 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
   else
     dg::launch_linear_simple(ex, dt, c->O, c->m.wo, c->X, c->Hs, M, d, qd);
   const void* hs = c->Hs;
+  if (c->m.n_experts) {
+    dg::launch_moe(ex, c->moe);
+    hs = c->Hs2;
+  }
   // inside a stream capture, only an "external" record becomes an event node
   if (c->cur_ev_start) DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start, ex.stream, cudaEventRecordExternal));
   if (dt == DG_BF16)
@@ -182,6 +193,8 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
     if (dbg->argmax) DG_CUDA_RET(cudaMemcpyAsync(dbg->argmax, c->am, M * sizeof(int32_t), cudaMemcpyDeviceToDevice, ex.stream));
     if (dbg->attn_out) DG_CUDA_RET(cudaMemcpyAsync(dbg->attn_out, c->O, (size_t)M * qd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
     if (dbg->hidden) DG_CUDA_RET(cudaMemcpyAsync(dbg->hidden, hs, (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->hidden_attn)
+      DG_CUDA_RET(cudaMemcpyAsync(dbg->hidden_attn, c->Hs, (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, ex.stream));
   }
   return DG_OK;
 }
@@ -285,6 +298,7 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   if (st != DG_OK) return st;
   DG_ARG(batch >= 1 && batch <= 4096, "batch must be in [1, 4096]");
   DG_ARG(canvas_len >= 1 && canvas_len <= 256, "canvas_len must be in [1, 256]");
+  if (model->n_experts) DG_UNSUP(batch * canvas_len <= 256, "the MoE FFN needs batch * canvas_len <= 256");
   DG_ARG(prefix_len && seeds, "prefix_len / seeds is NULL");
   for (int b = 0; b < batch; ++b) {
     DG_ARG(prefix_len[b] >= 0 && prefix_len[b] <= (1 << 24), "prefix_len out of range");
@@ -357,7 +371,8 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
     void* oo[1] = {c->Hs};
     const int no[1] = {model->d_model};
     dg::GemmTc gq = c->g_qkv, gw = c->g_wo;  // keep the bound buffers
-    if (!dg::lmhead_tc_prepare(c->Hs, model->lm_head, c->M, model->d_model, model->vocab, &c->tm_lm_a,
+    const void* lm_in = model->n_experts ? c->Hs2 : c->Hs;
+    if (!dg::lmhead_tc_prepare(lm_in, model->lm_head, c->M, model->d_model, model->vocab, &c->tm_lm_a,
                                &c->tm_lm_b) ||
         !dg::gemm_tc_prepare(&c->g_qkv, c->X, c->M, model->d_model, 3, wqkv, oqkv, nqkv, c->ex.sm_count) ||
         !dg::gemm_tc_prepare(&c->g_wo, c->O, c->M, qd, 1, wo, oo, no, c->ex.sm_count))
@@ -376,6 +391,12 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
     if (!dg::attn_tc_prepare(&c->attn, sh, c->Q, c->Kc, c->Vc, c->S.data(), c->pk.data(), c->pv.data(), c->O,
                              c->attn.part_o, c->attn.part_ml, c->attn_splits))
       return fail(DG_ERR_CUDA);
+    if (model->n_experts) {
+      dg::MoeShape ms{c->M, model->d_model, model->n_experts, model->top_k, model->n_shared, model->moe_inter};
+      if (!dg::moe_prepare(&c->moe, ms, c->Hs, c->Hs2, model->w_router, model->w_gate, model->w_up, model->w_down,
+                           c->moe_ws, c->ex.sm_count))
+        return fail(DG_ERR_UNSUPPORTED);
+    }
   }
 
   std::vector<dg::PrefixDesc> pd(batch);

@@ -20,7 +20,8 @@
 //              shared memory. The running maximum is only raised when the
 //              tile's maximum exceeds it by more than 8 (a factor 256), and
 //              then O and the running sum are rescaled in place; otherwise the
-//              stale maximum is kept (the result is the same ratio).
+//              stale maximum is kept (the result is the same ratio). The
+//              decision is per warp, since the TMEM accesses are collective.
 // With one split the rows are normalised and stored as bf16; with several,
 // unnormalised O and (max, sum) go to a partial buffer for attn_merge_kernel.
 #include <cstring>
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     uint8_t* prow = smem + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
-      if (!(ok = mbar_wait(&s_full[s], (i >> 1) & 1, p.err, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(&s_full[s], (i >> 1) & 1, p.err, abort_flag))) break;
       tc_fence_after();
       float x[128];
 #pragma unroll
@@ -260,12 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         mt = fmaxf(mt, x[c]);
       }
       if (i > 0) {  // PV_{i-1} done: O is stable and the P buffer is free
-        if (!(ok = mbar_wait(pv_done, (i - 1) & 1, p.err, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(pv_done, (i - 1) & 1, p.err, abort_flag))) break;
         tc_fence_after();
       }
-      if (mt > m_run + kRescaleThreshold) {
+      // The O rows live in TMEM and are rescaled with warp-collective
+      // tcgen05.ld/st, so the decision is taken per warp: when any row of the
+      // warp has outgrown its maximum by the threshold, every row of the warp
+      // moves its maximum up to its tile maximum (alpha = 1 where it stays).
+      if (__any_sync(0xffffffffu, mt > m_run + kRescaleThreshold)) {
+        const float m_new = fmaxf(m_run, mt);
         if (i > 0) {
-          const float alpha = ex2_approx(m_run - mt);
+          const float alpha = ex2_approx(m_run - m_new);
           l *= alpha;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -277,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
           tmem_st_wait();
         }
-        m_run = mt;
+        m_run = m_new;
       }
       // P = 2^(x - m_run) as bf16, 128B-swizzled K-major rows
 #pragma unroll
@@ -302,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (lane == 0) mbar_arrive(p_full);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n > 0 && mbar_wait(pv_done, (n - 1) & 1, p.err, abort_flag)) {
+    if (ok && n > 0 && mbar_wait_warp(pv_done, (n - 1) & 1, p.err, abort_flag)) {
       tc_fence_after();
       const int qrow = qt * kTile + r;
       const bool has_row = qrow < p.C;

@@ -49,6 +49,7 @@ struct Params {
   int nseg;
   Seg seg[3];
   const __nv_bfloat16* R;  // residual [M][ldo of segment 0] or null (single-segment use)
+  int out_f32;             // 1: outputs are f32 (no rounding; one split, no residual)
   int splits;              // K splits (gridDim.z)
   int ncols;               // total columns over the segments (partial buffer row length)
   float* part;             // [splits][M][ncols] f32 (splits > 1)
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int quad = warp & 3;
     const int row = m0 + quad * 32 + lane;
     const Seg sg = p.seg[seg];
-    const bool ok = mbar_wait(tfull, 0, p.err, abort_flag);
+    const bool ok = mbar_wait_warp(tfull, 0, p.err, abort_flag);
     tc_fence_after();
     if (ok) {
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
@@ -273,7 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
         if (row < p.M) {
-          if (p.splits == 1) {
+          if (p.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(sg.out) + (size_t)row * sg.ldo + n0 + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else if (p.splits == 1) {
             store_row32(sg.out + (size_t)row * sg.ldo + n0 + c * 32,
                         p.R ? p.R + (size_t)row * sg.ldo + n0 + c * 32 : nullptr, v);
           } else {  // this split's f32 partial; gemm_reduce_kernel sums the splits in order
@@ -401,6 +406,7 @@ void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual) {
     if (i < g.nseg) col0 += g.N[i];
   }
   p.R = static_cast<const __nv_bfloat16*>(residual);
+  p.out_f32 = g.out_f32;
   p.splits = g.splits;
   p.ncols = g.ncols;
   p.part = g.part;

@@ -90,6 +90,7 @@ void launch_lmhead_tc(Exec& ex, const CUtensorMap& tmA, const CUtensorMap& tmB, 
 struct alignas(64) GemmTc {
   unsigned char maps[4 * 128];  // CUtensorMap for A and each W_i
   int M = 0, K = 0, nseg = 0, tiles = 0, bn = 64, splits = 1, ncols = 0;
+  int out_f32 = 0;               // f32 outputs (set after prepare; requires splits == 1)
   void* out[3] = {nullptr, nullptr, nullptr};
   int N[3] = {0, 0, 0};
   float* part = nullptr;         // split-K partials [splits][M][ncols]
@@ -126,6 +127,32 @@ bool attn_tc_prepare(AttnTc* at, const AttnShape& sh, const void* Q, const void*
                      const int32_t* S, const void* const* pk, const void* const* pv, void* O, float* part_o,
                      float* part_ml, int splits);
 void launch_attn_tc(Exec& ex, const AttnTc& at);
+
+// MoE FFN (bf16): router GEMM, routing, gather, expert gate/up and down GEMMs,
+// combine; all buffers in one workspace region of moe_workspace_bytes().
+struct MoeShape {
+  int M, d, E, topk, nsh, I;
+};
+struct MoeTc {
+  MoeShape s{};
+  const void* hs = nullptr;  // residual stream in [M][d]
+  void* hs_out = nullptr;    // residual stream out [M][d]
+  float* logits = nullptr;   // [M][E]
+  float* gate = nullptr;     // [M][topk]
+  int* pos = nullptr;        // [M][topk + nsh]
+  int* off = nullptr;        // [E + nsh + 1]
+  int* pair_tok = nullptr;   // [R]
+  void* xg = nullptr;        // [R][d] bf16
+  void* act = nullptr;       // [R][I] bf16
+  float* y = nullptr;        // [R][d]
+  GemmTc router;
+  alignas(64) unsigned char maps_gateup[3 * 128];
+  alignas(64) unsigned char maps_down[3 * 128];
+};
+size_t moe_workspace_bytes(const MoeShape& s);
+bool moe_prepare(MoeTc* mt, const MoeShape& s, const void* hs, void* hs_out, const void* w_router,
+                 const void* w_gate, const void* w_up, const void* w_down, void* ws, int sm_count);
+void launch_moe(Exec& ex, const MoeTc& mt);
 
 // ---- canvas bookkeeping
 struct CanvasState {
@@ -176,6 +203,8 @@ struct dg_ctx {
   dg::GemmTc g_qkv, g_wo;
   dg::AttnTc attn;
   int attn_splits = 1;
+  dg::MoeTc moe;
+  void* moe_ws = nullptr;
 
   int launches = 0;  // kernels queued by the last denoise step
 

@@ -210,7 +210,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     for (int t = 0; t < n_tiles; ++t) {
       const int gt = g0 + t * kMaxGran;
       const int ncol = min(kMaxGran, g1 - gt) * kGranule;
-      if (!mbar_wait(tfull, tph, p.err, abort_flag)) break;
+      if (!mbar_wait_warp(tfull, tph, p.err, abort_flag)) break;
       tc_fence_after();
       if (half < halves) {
         for (int c0 = 0; c0 < ncol; c0 += 32) {

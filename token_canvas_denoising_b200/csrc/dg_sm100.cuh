@@ -80,6 +80,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
   }
 }
 
+// mbar_wait for warps that go on to warp-collective tcgen05.ld / tcgen05.st
+// (.sync.aligned: every lane must execute them together): the result is the
+// same in every lane, true only if the wait succeeded in all of them.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* err, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, err, abort));
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

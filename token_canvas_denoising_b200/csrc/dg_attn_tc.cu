@@ -40,13 +40,16 @@ constexpr int kTile = 128;
 constexpr int kAtom = 128 * 128;       // 128 rows x 128 B = 16 KB
 constexpr int kMatBytes = 2 * kAtom;   // a 128 x 128 bf16 tile = 32 KB
 constexpr int kStages = 2;
-// smem: Q | K0 V0 | K1 V1 | P
+// smem: Q | K0 V0 | K1 V1 | P0 | P1
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kMatBytes;
 constexpr int kOffP = kOffKV + kStages * 2 * kMatBytes;
-constexpr int kSmemBytes = kOffP + kMatBytes + 1024 + 256;
+constexpr int kOffBar = kOffP + 2 * kMatBytes;
+constexpr int kSmemBytes = kOffBar + 1024 + 256;
+static_assert(kSmemBytes <= 232448, "attention tile exceeds the opt-in shared memory of a CTA");
 constexpr int kMaxReq = 8;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
+constexpr int kAhead = 4;                 // prompt-prefix tiles prefetched into L2 ahead of their load
 
 struct Maps {
   CUtensorMap q;    // [B*C][Hq*h]
@@ -69,6 +72,31 @@ struct Params {
   int* err;
 };
 
+// P row of one tile: p = 2^(x scale - m) as bf16, written 128B-swizzled
+// K-major, row sums accumulated over 8 chains.
+__device__ __forceinline__ void store_p_row(const float (&x)[128], float scale, float neg_m, uint8_t* prow, int r,
+                                            float (&ls)[8]) {
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      uint4 w;
+      __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float t0 = fmaf(x[a * 64 + ch * 8 + 2 * e], scale, neg_m);
+        const float t1 = fmaf(x[a * 64 + ch * 8 + 2 * e + 1], scale, neg_m);
+        const float p0 = ex2_approx(t0);
+        const float p1 = ex2_approx(t1);
+        ls[2 * e] += p0;
+        ls[2 * e + 1] += p1;
+        w2[e] = __floats2bfloat162_rn(p0, p1);
+      }
+      *reinterpret_cast<uint4*>(prow + a * kAtom + ((ch ^ (r & 7)) << 4)) = w;
+    }
+  }
+}
+
 __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
   // K-major 128-row operand with 128 columns of K split into two 64-wide atoms
   return umma_desc_sw128(base + (kk >> 2) * kAtom + (kk & 3) * 32, 16, 1024);
@@ -77,16 +105,17 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Maps maps, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffP + kMatBytes);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bar + 0;
   uint64_t* k_full = bar + 1;      // [2]
   uint64_t* v_full = bar + 3;      // [2]
-  uint64_t* kv_empty = bar + 5;    // [2]
-  uint64_t* s_full = bar + 7;      // [2]
-  uint64_t* s_free = bar + 9;      // [2]
-  uint64_t* p_full = bar + 11;
-  uint64_t* pv_done = bar + 12;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 13);
+  uint64_t* k_empty = bar + 5;     // [2] QK_i done: K slot i & 1 free
+  uint64_t* v_empty = bar + 7;     // [2] PV_i done: V slot i & 1 free
+  uint64_t* s_full = bar + 9;      // [2]
+  uint64_t* s_free = bar + 11;     // [2]
+  uint64_t* p_full = bar + 13;     // [2] P_i written to buffer i & 1
+  uint64_t* pv_done = bar + 15;    // [2] PV_i (reading P buffer i & 1) complete
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,12 +138,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -133,36 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
-      bool issued_q = false;
-      bool issued[2] = {false, false};
-      uint32_t iph[2] = {0, 0};
-      // the prompt prefix is an input of the step: its first tiles may be
-      // fetched before the predecessor kernels are done
-      int pre = 0;
-      while (pre < 2 && pre < n && t0 + pre < nps) {
-        const int s = pre;
-        uint8_t* kb = smem + kOffKV + s * 2 * kMatBytes;
-        mbar_arrive_expect_tx(&k_full[s], kMatBytes);
-        for (int a = 0; a < 2; ++a) tma_load_2d(kb + a * kAtom, &maps.pk[lb], &k_full[s], g * 128 + a * 64, (t0 + pre) * kTile, pol);
-        mbar_arrive_expect_tx(&v_full[s], kMatBytes);
-        for (int a = 0; a < 2; ++a)
-          tma_load_2d(kb + kMatBytes + a * kAtom, &maps.pv[lb], &v_full[s], g * 128 + a * 64, (t0 + pre) * kTile, pol);
-        issued[s] = true;
-        iph[s] = 0;
-        ++pre;
-      }
-      griddep_wait();
-      mbar_arrive_expect_tx(q_full, kMatBytes);
-      for (int a = 0; a < 2; ++a)
-        tma_load_2d(smem + kOffQ + a * kAtom, &maps.q, q_full, qh * 128 + a * 64, b * p.C + qt * kTile, pol);
-      issued_q = true;
-      for (int i = pre; i < n && !*abort_flag; ++i) {
-        const int s = i & 1;
-        if (i >= 2 && !mbar_wait(&kv_empty[s], ((i >> 1) - 1) & 1, p.err, abort_flag)) break;
+      // tile i: K and V rows [y, y + 128) of the prompt prefix or of the canvas
+      auto tile_src = [&](int i, const CUtensorMap*& mk, const CUtensorMap*& mv, int& y) {
         const int j = t0 + i;
-        const CUtensorMap* mk;
-        const CUtensorMap* mv;
-        int y;
         if (j < nps) {
           mk = &maps.pk[lb];
           mv = &maps.pv[lb];
@@ -172,22 +175,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           mv = &maps.vc;
           y = b * p.C + (j - nps) * kTile;
         }
-        uint8_t* kb = smem + kOffKV + s * 2 * kMatBytes;
-        uint8_t* vb = kb + kMatBytes;
-        mbar_arrive_expect_tx(&k_full[s], kMatBytes);
-        for (int a = 0; a < 2; ++a) tma_load_2d(kb + a * kAtom, mk, &k_full[s], g * 128 + a * 64, y, pol);
-        mbar_arrive_expect_tx(&v_full[s], kMatBytes);
-        for (int a = 0; a < 2; ++a) tma_load_2d(vb + a * kAtom, mv, &v_full[s], g * 128 + a * 64, y, pol);
-        issued[s] = true;
-        iph[s] = (i >> 1) & 1;
-      }
-      if (*abort_flag) {  // drain this CTA's own copies
-        if (issued_q) mbar_wait(q_full, 0, p.err, nullptr);
-        for (int s = 0; s < 2; ++s)
-          if (issued[s]) {
-            mbar_wait(&k_full[s], iph[s], p.err, nullptr);
-            mbar_wait(&v_full[s], iph[s], p.err, nullptr);
+      };
+      auto load_k = [&](int i) {
+        const CUtensorMap *mk, *mv;
+        int y;
+        tile_src(i, mk, mv, y);
+        uint8_t* kb = smem + kOffKV + (i & 1) * 2 * kMatBytes;
+        mbar_arrive_expect_tx(&k_full[i & 1], kMatBytes);
+        for (int a = 0; a < 2; ++a) tma_load_2d(kb + a * kAtom, mk, &k_full[i & 1], g * 128 + a * 64, y, pol);
+      };
+      auto load_v = [&](int i) {
+        const CUtensorMap *mk, *mv;
+        int y;
+        tile_src(i, mk, mv, y);
+        uint8_t* vb = smem + kOffKV + (i & 1) * 2 * kMatBytes + kMatBytes;
+        mbar_arrive_expect_tx(&v_full[i & 1], kMatBytes);
+        for (int a = 0; a < 2; ++a) tma_load_2d(vb + a * kAtom, mv, &v_full[i & 1], g * 128 + a * 64, y, pol);
+      };
+      // prompt-prefix tiles further ahead are pulled into L2 early
+      auto prefetch = [&](int i) {
+        if (i < n && t0 + i < nps) {
+          for (int a = 0; a < 2; ++a) {
+            tma_prefetch_2d(&maps.pk[lb], g * 128 + a * 64, (t0 + i) * kTile);
+            tma_prefetch_2d(&maps.pv[lb], g * 128 + a * 64, (t0 + i) * kTile);
           }
+        }
+      };
+      int nk = 0, nv = 0;  // next K tile and next V tile to load
+      // the prompt prefix is an input of the step: its first tiles may be
+      // fetched before the predecessor kernels are done
+      while (nk < 2 && nk < n && t0 + nk < nps) {
+        load_k(nk);
+        load_v(nk);
+        ++nk;
+        ++nv;
+      }
+      for (int i = nk; i < nk + kAhead; ++i) prefetch(i);
+      griddep_wait();
+      mbar_arrive_expect_tx(q_full, kMatBytes);
+      for (int a = 0; a < 2; ++a)
+        tma_load_2d(smem + kOffQ + a * kAtom, &maps.q, q_full, qh * 128 + a * 64, b * p.C + qt * kTile, pol);
+      // K runs one tile ahead of V: a K slot frees when its QK completes, a V
+      // slot only when its PV does.
+      while (nv < n && !*abort_flag) {
+        if (nk < n && nk <= nv + 1) {
+          if (nk >= 2 && !mbar_wait(&k_empty[nk & 1], ((nk >> 1) - 1) & 1, p.err, abort_flag)) break;
+          load_k(nk);
+          prefetch(nk + kAhead);
+          ++nk;
+        } else {
+          if (nv >= 2 && !mbar_wait(&v_empty[nv & 1], ((nv >> 1) - 1) & 1, p.err, abort_flag)) break;
+          load_v(nv);
+          ++nv;
+        }
+      }
+      if (*abort_flag) {  // drain this CTA's own copies: the last load of each slot
+        mbar_wait(q_full, 0, p.err, nullptr);
+        for (int i = nk - 2; i < nk; ++i)
+          if (i >= 0) mbar_wait(&k_full[i & 1], (i >> 1) & 1, p.err, nullptr);
+        for (int i = nv - 2; i < nv; ++i)
+          if (i >= 0) mbar_wait(&v_full[i & 1], (i >> 1) & 1, p.err, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -209,22 +256,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ss(tmem + s * 128, kdesc(qbase, kk), kdesc(kbase, kk), id_qk, kk != 0);
         mma_commit(&s_full[s]);
+        mma_commit(&k_empty[s]);
         return true;
       };
       if (ok && n > 0) ok = issue_qk(0);
       for (int i = 0; ok && i < n; ++i) {
         if (i + 1 < n && !(ok = issue_qk(i + 1))) break;
         const int s = i & 1;
-        if (!mbar_wait(p_full, i & 1, p.err, abort_flag)) break;
+        if (!mbar_wait(&p_full[s], (i >> 1) & 1, p.err, abort_flag)) break;
         if (!mbar_wait(&v_full[s], (i >> 1) & 1, p.err, abort_flag)) break;
         tc_fence_after();
         const uint32_t vbase = smem_u32(smem + kOffKV + s * 2 * kMatBytes + kMatBytes);
+        const uint32_t pb = pbase + s * kMatBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem_o, kdesc(pbase, kk), umma_desc_sw128(vbase + kk * 2048, kAtom, 1024), id_pv,
+          mma_bf16_ss(tmem_o, kdesc(pb, kk), umma_desc_sw128(vbase + kk * 2048, kAtom, 1024), id_pv,
                       (i | kk) != 0);
-        mma_commit(pv_done);
-        mma_commit(&kv_empty[s]);
+        mma_commit(&pv_done[s]);
+        mma_commit(&v_empty[s]);
       }
     }
   } else {
@@ -235,18 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow = smem + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
+    uint8_t* prow0 = smem + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
       if (!(ok = mbar_wait_warp(&s_full[s], (i >> 1) & 1, p.err, abort_flag))) break;
       tc_fence_after();
       float x[128];
+      {
+        uint32_t u[128];
+        tmem_ld128_sync(tmem + lane_off + s * 128, u);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t u[32];
-        tmem_ld32_sync(tmem + lane_off + s * 128 + c * 32, u);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
       }
       tc_fence_before();
       __syncwarp();
@@ -254,23 +302,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // keys of this tile that exist
       const int j = t0 + i;
       const int valid = (j < nps) ? min(kTile, S - j * kTile) : min(kTile, p.C - (j - nps) * kTile);
-      float mt = -INFINITY;
+      if (valid < kTile) {  // ragged last tile (uniform over the CTA)
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = (c < valid) ? x[c] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, x[c]);
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) x[c] = -INFINITY;
       }
-      if (i > 0) {  // PV_{i-1} done: O is stable and the P buffer is free
-        if (!(ok = mbar_wait_warp(pv_done, (i - 1) & 1, p.err, abort_flag))) break;
-        tc_fence_after();
-      }
+      // row maximum over 8 independent chains (short dependency chains)
+      float mx[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = x[c];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
+      const float mt = mx[0] * p.scale_log2;  // the scale is positive: maximum of the scaled scores
       // The O rows live in TMEM and are rescaled with warp-collective
       // tcgen05.ld/st, so the decision is taken per warp: when any row of the
       // warp has outgrown its maximum by the threshold, every row of the warp
       // moves its maximum up to its tile maximum (alpha = 1 where it stays).
       if (__any_sync(0xffffffffu, mt > m_run + kRescaleThreshold)) {
         const float m_new = fmaxf(m_run, mt);
-        if (i > 0) {
+        if (i > 0) {  // O must hold PV_{i-1} before it is scaled
+          if (!(ok = mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, p.err, abort_flag))) break;
+          tc_fence_after();
           const float alpha = ex2_approx(m_run - m_new);
           l *= alpha;
 #pragma unroll
@@ -285,30 +341,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         m_run = m_new;
       }
-      // P = 2^(x - m_run) as bf16, 128B-swizzled K-major rows
-#pragma unroll
-      for (int a = 0; a < 2; ++a) {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 w;
-          __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2_approx(x[a * 64 + ch * 8 + 2 * e] - m_run);
-            const float p1 = ex2_approx(x[a * 64 + ch * 8 + 2 * e + 1] - m_run);
-            l += p0 + p1;
-            w2[e] = __floats2bfloat162_rn(p0, p1);
-          }
-          *reinterpret_cast<uint4*>(prow + a * kAtom + ((ch ^ (r & 7)) << 4)) = w;
-        }
+      // P buffer s was last read by PV_{i-2}
+      if (i >= 2) {
+        if (!(ok = mbar_wait_warp(&pv_done[s], ((i >> 1) - 1) & 1, p.err, abort_flag))) break;
       }
+      // P = 2^(x scale - m_run) as bf16, 128B-swizzled K-major rows
+      uint8_t* prow = prow0 + s * kMatBytes;
+      const float neg_m = -m_run;
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      store_p_row(x, p.scale_log2, neg_m, prow, r, ls);
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       fence_async_shared();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[s]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n > 0 && mbar_wait_warp(pv_done, (n - 1) & 1, p.err, abort_flag)) {
+    if (ok && n > 0 && mbar_wait_warp(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, p.err, abort_flag)) {
       tc_fence_after();
       const int qrow = qt * kTile + r;
       const bool has_row = qrow < p.C;

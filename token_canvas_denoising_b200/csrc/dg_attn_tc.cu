@@ -9,19 +9,25 @@
 //
 // CTA work item: (request b, query head q, 128-query tile, KV split). The KV
 // sequence is walked in 128-key tiles (prefix tiles from the request's own
-// tensor map, then canvas tiles), with a 2-stage TMA pipeline for K and V.
-//   warp 0   : TMA producer (Q once, then K_j and V_j per tile)
+// tensor map, then canvas tiles) through 3-slot TMA rings for K and for V.
+//   warp 0   : TMA producer: Q once; K tiles one ahead of V tiles (a K slot
+//              frees when its QK completes, a V slot when its PV does);
+//              prompt-prefix tiles a few tiles ahead are prefetched into L2
 //   warp 1   : TMEM allocator and MMA issuer: S_j = Q K_j^T (M=N=128, K=128)
 //              into one of two TMEM score buffers, then O += P_j V_j (V as an
-//              MN-major operand) into the TMEM output accumulator
-//   warps 2-5: softmax, one query row per thread: read S_j from TMEM, mask the
+//              MN-major operand) into the TMEM output accumulator. Q and P are
+//              A operands read from TMEM, so shared memory only feeds K and V
+//              (the tile's operand traffic through shared memory halves).
+//   warps 2-5: softmax, one query row per thread: copy the Q row from shared
+//              memory into TMEM once; per tile read S_j from TMEM, mask the
 //              keys past the tile's end, exponentiate in base 2 against a
-//              running maximum, write P_j (bf16, 128B-swizzled K-major) to
-//              shared memory. The running maximum is only raised when the
-//              tile's maximum exceeds it by more than 8 (a factor 256), and
-//              then O and the running sum are rescaled in place; otherwise the
-//              stale maximum is kept (the result is the same ratio). The
-//              decision is per warp, since the TMEM accesses are collective.
+//              running maximum, write P_j (bf16 pairs) into TMEM. The running
+//              maximum is only raised when the tile's maximum exceeds it by
+//              more than 8 (a factor 256), and then O and the running sum are
+//              rescaled in place; otherwise the stale maximum is kept (the
+//              result is the same ratio). The decision is per warp, since the
+//              TMEM accesses are collective.
+// TMEM columns: S0 [0,128) | S1 [128,256) | O [256,384) | Q [384,448) | P [448,512).
 // With one split the rows are normalised and stored as bf16; with several,
 // unnormalised O and (max, sum) go to a partial buffer for attn_merge_kernel.
 #include <cstring>
@@ -39,17 +45,20 @@ constexpr int kThreads = 192;
 constexpr int kTile = 128;
 constexpr int kAtom = 128 * 128;       // 128 rows x 128 B = 16 KB
 constexpr int kMatBytes = 2 * kAtom;   // a 128 x 128 bf16 tile = 32 KB
-constexpr int kStages = 2;
-// smem: Q | K0 V0 | K1 V1 | P0 | P1
+constexpr int kSlots = 3;              // K ring and V ring depth
+// smem: Q | K0 K1 K2 | V0 V1 V2 | barriers. The dynamic shared window starts
+// 1024-aligned (after the CTA's reserved 1 KB); the kernel checks this
+// instead of reserving alignment slack.
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kMatBytes;
-constexpr int kOffP = kOffKV + kStages * 2 * kMatBytes;
-constexpr int kOffBar = kOffP + 2 * kMatBytes;
-constexpr int kSmemBytes = kOffBar + 1024 + 256;
+constexpr int kOffK = kMatBytes;
+constexpr int kOffV = kOffK + kSlots * kMatBytes;
+constexpr int kOffBar = kOffV + kSlots * kMatBytes;
+constexpr int kSmemBytes = kOffBar + 256;
 static_assert(kSmemBytes <= 232448, "attention tile exceeds the opt-in shared memory of a CTA");
 constexpr int kMaxReq = 8;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 constexpr int kAhead = 4;                 // prompt-prefix tiles prefetched into L2 ahead of their load
+constexpr uint32_t kColO = 256, kColQ = 384, kColP = 448;
 
 struct Maps {
   CUtensorMap q;    // [B*C][Hq*h]
@@ -72,50 +81,30 @@ struct Params {
   int* err;
 };
 
-// P row of one tile: p = 2^(x scale - m) as bf16, written 128B-swizzled
-// K-major, row sums accumulated over 8 chains.
-__device__ __forceinline__ void store_p_row(const float (&x)[128], float scale, float neg_m, uint8_t* prow, int r,
-                                            float (&ls)[8]) {
-#pragma unroll
-  for (int a = 0; a < 2; ++a) {
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      uint4 w;
-      __nv_bfloat162* w2 = reinterpret_cast<__nv_bfloat162*>(&w);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float t0 = fmaf(x[a * 64 + ch * 8 + 2 * e], scale, neg_m);
-        const float t1 = fmaf(x[a * 64 + ch * 8 + 2 * e + 1], scale, neg_m);
-        const float p0 = ex2_approx(t0);
-        const float p1 = ex2_approx(t1);
-        ls[2 * e] += p0;
-        ls[2 * e + 1] += p1;
-        w2[e] = __floats2bfloat162_rn(p0, p1);
-      }
-      *reinterpret_cast<uint4*>(prow + a * kAtom + ((ch ^ (r & 7)) << 4)) = w;
-    }
-  }
-}
-
 __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
   // K-major 128-row operand with 128 columns of K split into two 64-wide atoms
   return umma_desc_sw128(base + (kk >> 2) * kAtom + (kk & 3) * 32, 16, 1024);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Maps maps, Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {  // SW128 tiles need 1024-byte alignment (uniform: no TMEM held yet)
+    if (threadIdx.x == 0) set_error(p.err, kDevBadAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* q_full = bar + 0;
-  uint64_t* k_full = bar + 1;      // [2]
-  uint64_t* v_full = bar + 3;      // [2]
-  uint64_t* k_empty = bar + 5;     // [2] QK_i done: K slot i & 1 free
-  uint64_t* v_empty = bar + 7;     // [2] PV_i done: V slot i & 1 free
-  uint64_t* s_full = bar + 9;      // [2]
-  uint64_t* s_free = bar + 11;     // [2]
-  uint64_t* p_full = bar + 13;     // [2] P_i written to buffer i & 1
-  uint64_t* pv_done = bar + 15;    // [2] PV_i (reading P buffer i & 1) complete
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 17);
+  uint64_t* q_full = bar + 0;      // Q tile landed in shared memory
+  uint64_t* q_tmem = bar + 1;      // Q copied into TMEM (4 softmax warps)
+  uint64_t* k_full = bar + 2;      // [3]
+  uint64_t* v_full = bar + 5;      // [3]
+  uint64_t* k_empty = bar + 8;     // [3] QK_i done: K slot i % 3 free
+  uint64_t* v_empty = bar + 11;    // [3] PV_i done: V slot i % 3 free
+  uint64_t* s_full = bar + 14;     // [2] S_i in TMEM buffer i & 1
+  uint64_t* s_free = bar + 16;     // [2] S buffer read by the softmax (4 warps)
+  uint64_t* p_full = bar + 18;     // P_i in TMEM (4 warps)
+  uint64_t* pv_done = bar + 19;    // PV_i complete: O stable, P columns free
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,16 +124,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(q_tmem, 4);
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
     }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -157,7 +149,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_o = tmem + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -180,17 +171,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const CUtensorMap *mk, *mv;
         int y;
         tile_src(i, mk, mv, y);
-        uint8_t* kb = smem + kOffKV + (i & 1) * 2 * kMatBytes;
-        mbar_arrive_expect_tx(&k_full[i & 1], kMatBytes);
-        for (int a = 0; a < 2; ++a) tma_load_2d(kb + a * kAtom, mk, &k_full[i & 1], g * 128 + a * 64, y, pol);
+        uint8_t* kb = smem + kOffK + (i % kSlots) * kMatBytes;
+        mbar_arrive_expect_tx(&k_full[i % kSlots], kMatBytes);
+        for (int a = 0; a < 2; ++a) tma_load_2d(kb + a * kAtom, mk, &k_full[i % kSlots], g * 128 + a * 64, y, pol);
       };
       auto load_v = [&](int i) {
         const CUtensorMap *mk, *mv;
         int y;
         tile_src(i, mk, mv, y);
-        uint8_t* vb = smem + kOffKV + (i & 1) * 2 * kMatBytes + kMatBytes;
-        mbar_arrive_expect_tx(&v_full[i & 1], kMatBytes);
-        for (int a = 0; a < 2; ++a) tma_load_2d(vb + a * kAtom, mv, &v_full[i & 1], g * 128 + a * 64, y, pol);
+        uint8_t* vb = smem + kOffV + (i % kSlots) * kMatBytes;
+        mbar_arrive_expect_tx(&v_full[i % kSlots], kMatBytes);
+        for (int a = 0; a < 2; ++a) tma_load_2d(vb + a * kAtom, mv, &v_full[i % kSlots], g * 128 + a * 64, y, pol);
       };
       // prompt-prefix tiles further ahead are pulled into L2 early
       auto prefetch = [&](int i) {
@@ -204,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       int nk = 0, nv = 0;  // next K tile and next V tile to load
       // the prompt prefix is an input of the step: its first tiles may be
       // fetched before the predecessor kernels are done
-      while (nk < 2 && nk < n && t0 + nk < nps) {
+      while (nk < kSlots && nk < n && t0 + nk < nps) {
         load_k(nk);
         load_v(nk);
         ++nk;
@@ -215,26 +206,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_arrive_expect_tx(q_full, kMatBytes);
       for (int a = 0; a < 2; ++a)
         tma_load_2d(smem + kOffQ + a * kAtom, &maps.q, q_full, qh * 128 + a * 64, b * p.C + qt * kTile, pol);
-      // K runs one tile ahead of V: a K slot frees when its QK completes, a V
-      // slot only when its PV does.
+      // K runs one tile ahead of V
       while (nv < n && !*abort_flag) {
         if (nk < n && nk <= nv + 1) {
-          if (nk >= 2 && !mbar_wait(&k_empty[nk & 1], ((nk >> 1) - 1) & 1, p.err, abort_flag)) break;
+          if (nk >= kSlots && !mbar_wait(&k_empty[nk % kSlots], ((nk / kSlots) - 1) & 1, p.err, abort_flag)) break;
           load_k(nk);
           prefetch(nk + kAhead);
           ++nk;
         } else {
-          if (nv >= 2 && !mbar_wait(&v_empty[nv & 1], ((nv >> 1) - 1) & 1, p.err, abort_flag)) break;
+          if (nv >= kSlots && !mbar_wait(&v_empty[nv % kSlots], ((nv / kSlots) - 1) & 1, p.err, abort_flag)) break;
           load_v(nv);
           ++nv;
         }
       }
       if (*abort_flag) {  // drain this CTA's own copies: the last load of each slot
         mbar_wait(q_full, 0, p.err, nullptr);
-        for (int i = nk - 2; i < nk; ++i)
-          if (i >= 0) mbar_wait(&k_full[i & 1], (i >> 1) & 1, p.err, nullptr);
-        for (int i = nv - 2; i < nv; ++i)
-          if (i >= 0) mbar_wait(&v_full[i & 1], (i >> 1) & 1, p.err, nullptr);
+        for (int i = nk - kSlots; i < nk; ++i)
+          if (i >= 0) mbar_wait(&k_full[i % kSlots], (i / kSlots) & 1, p.err, nullptr);
+        for (int i = nv - kSlots; i < nv; ++i)
+          if (i >= 0) mbar_wait(&v_full[i % kSlots], (i / kSlots) & 1, p.err, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -243,37 +233,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(128, 128, false);
       const uint32_t id_pv = idesc_bf16_f32(128, 128, true);
-      const uint32_t qbase = smem_u32(smem + kOffQ);
-      const uint32_t pbase = smem_u32(smem + kOffP);
-      bool ok = mbar_wait(q_full, 0, p.err, abort_flag);
+      bool ok = mbar_wait(q_tmem, 0, p.err, abort_flag);
       auto issue_qk = [&](int i) -> bool {
-        const int s = i & 1;
-        if (!mbar_wait(&k_full[s], (i >> 1) & 1, p.err, abort_flag)) return false;
+        const int s = i & 1, slot = i % kSlots;
+        if (!mbar_wait(&k_full[slot], (i / kSlots) & 1, p.err, abort_flag)) return false;
         if (i >= 2 && !mbar_wait(&s_free[s], ((i >> 1) - 1) & 1, p.err, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t kbase = smem_u32(smem + kOffKV + s * 2 * kMatBytes);
+        const uint32_t kbase = smem_u32(smem + kOffK + slot * kMatBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + s * 128, kdesc(qbase, kk), kdesc(kbase, kk), id_qk, kk != 0);
+          mma_bf16_ts(tmem + s * 128, tmem + kColQ + kk * 8, kdesc(kbase, kk), id_qk, kk != 0);
         mma_commit(&s_full[s]);
-        mma_commit(&k_empty[s]);
+        mma_commit(&k_empty[slot]);
         return true;
       };
       if (ok && n > 0) ok = issue_qk(0);
       for (int i = 0; ok && i < n; ++i) {
         if (i + 1 < n && !(ok = issue_qk(i + 1))) break;
-        const int s = i & 1;
-        if (!mbar_wait(&p_full[s], (i >> 1) & 1, p.err, abort_flag)) break;
-        if (!mbar_wait(&v_full[s], (i >> 1) & 1, p.err, abort_flag)) break;
+        const int slot = i % kSlots;
+        if (!mbar_wait(p_full, i & 1, p.err, abort_flag)) break;
+        if (!mbar_wait(&v_full[slot], (i / kSlots) & 1, p.err, abort_flag)) break;
         tc_fence_after();
-        const uint32_t vbase = smem_u32(smem + kOffKV + s * 2 * kMatBytes + kMatBytes);
-        const uint32_t pb = pbase + s * kMatBytes;
+        const uint32_t vbase = smem_u32(smem + kOffV + slot * kMatBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem_o, kdesc(pb, kk), umma_desc_sw128(vbase + kk * 2048, kAtom, 1024), id_pv,
+          mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, umma_desc_sw128(vbase + kk * 2048, kAtom, 1024), id_pv,
                       (i | kk) != 0);
-        mma_commit(&pv_done[s]);
-        mma_commit(&v_empty[s]);
+        mma_commit(pv_done);
+        mma_commit(&v_empty[slot]);
       }
     }
   } else {
@@ -283,9 +270,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int r = quad * 32 + lane;  // query row within the tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     float m_run = -INFINITY, l = 0.f;
-    bool ok = true;
-    uint8_t* prow0 = smem + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
-    for (int i = 0; i < n; ++i) {
+    // Q row into TMEM columns [384, 448): 16-byte chunk c of swizzle atom a
+    // holds head dims a*64 + c*8 .. +7, i.e. columns a*32 + c*4 .. +3
+    bool ok = mbar_wait_warp(q_full, 0, p.err, abort_flag);
+    if (ok) {
+      const uint8_t* qrow = smem + kOffQ + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        uint32_t u[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qrow + a * kAtom + ((c ^ (r & 7)) << 4));
+          u[c * 4 + 0] = v.x;
+          u[c * 4 + 1] = v.y;
+          u[c * 4 + 2] = v.z;
+          u[c * 4 + 3] = v.w;
+        }
+        tmem_st32(tmem + lane_off + kColQ + a * 32, u);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_tmem);
+    }
+    for (int i = 0; ok && i < n; ++i) {
       const int s = i & 1;
       if (!(ok = mbar_wait_warp(&s_full[s], (i >> 1) & 1, p.err, abort_flag))) break;
       tc_fence_after();
@@ -322,42 +330,59 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // tcgen05.ld/st, so the decision is taken per warp: when any row of the
       // warp has outgrown its maximum by the threshold, every row of the warp
       // moves its maximum up to its tile maximum (alpha = 1 where it stays).
-      if (__any_sync(0xffffffffu, mt > m_run + kRescaleThreshold)) {
+      const bool rescale = __any_sync(0xffffffffu, mt > m_run + kRescaleThreshold);
+      float alpha = 1.f;
+      if (rescale) {
         const float m_new = fmaxf(m_run, mt);
-        if (i > 0) {  // O must hold PV_{i-1} before it is scaled
-          if (!(ok = mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, p.err, abort_flag))) break;
-          tc_fence_after();
-          const float alpha = ex2_approx(m_run - m_new);
-          l *= alpha;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t u[32];
-            tmem_ld32_sync(tmem_o + lane_off + c * 32, u);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(tmem_o + lane_off + c * 32, u);
-          }
-          tmem_st_wait();
-        }
+        alpha = ex2_approx(m_run - m_new);
         m_run = m_new;
       }
-      // P buffer s was last read by PV_{i-2}
-      if (i >= 2) {
-        if (!(ok = mbar_wait_warp(&pv_done[s], ((i >> 1) - 1) & 1, p.err, abort_flag))) break;
-      }
-      // P = 2^(x scale - m_run) as bf16, 128B-swizzled K-major rows
-      uint8_t* prow = prow0 + s * kMatBytes;
-      const float neg_m = -m_run;
+      // P = 2^(x scale - m_run) as bf16 pairs, row sum over 8 chains
+      uint32_t pk[64];
       float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      store_p_row(x, p.scale_log2, neg_m, prow, r, ls);
+      const float neg_m = -m_run;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2_approx(fmaf(x[2 * c], p.scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(x[2 * c + 1], p.scale_log2, neg_m));
+        ls[(2 * c) & 7] += p0;
+        ls[(2 * c + 1) & 7] += p1;
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      // PV_{i-1} complete: O holds it (for the rescale) and the P columns are free
+      if (i > 0) {
+        if (!(ok = mbar_wait_warp(pv_done, (i - 1) & 1, p.err, abort_flag))) break;
+        tc_fence_after();
+      }
+      if (rescale && i > 0) {
+        l *= alpha;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t u[32];
+          tmem_ld32_sync(tmem + lane_off + kColO + c * 32, u);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+          tmem_st32(tmem + lane_off + kColO + c * 32, u);
+        }
+      }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      fence_async_shared();
+      {
+        uint32_t u[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) u[e] = pk[e];
+        tmem_st32(tmem + lane_off + kColP, u);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) u[e] = pk[32 + e];
+        tmem_st32(tmem + lane_off + kColP + 32, u);
+      }
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[s]);
+      if (lane == 0) mbar_arrive(p_full);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n > 0 && mbar_wait_warp(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, p.err, abort_flag)) {
+    if (ok && n > 0 && mbar_wait_warp(pv_done, (n - 1) & 1, p.err, abort_flag)) {
       tc_fence_after();
       const int qrow = qt * kTile + r;
       const bool has_row = qrow < p.C;
@@ -366,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t u[32];
-        tmem_ld32_sync(tmem_o + lane_off + c * 32, u);
+        tmem_ld32_sync(tmem + lane_off + kColO + c * 32, u);
         if (!has_row) continue;
         if (p.splits == 1) {
           uint4* dst = reinterpret_cast<uint4*>(p.O + grow * p.Hq * 128 + qh * 128 + c * 32);

@@ -16,6 +16,7 @@ enum DeviceError : int {
   kDevNanEntropy = 2,    // entropy not finite
   kDevWaitTimeout = 3,   // a bounded mbarrier wait gave up
   kDevBadShape = 4,      // a kernel was launched on shapes it does not support
+  kDevBadAlign = 5,      // shared memory not aligned as a kernel's tile layout needs
 };
 
 __device__ __forceinline__ void set_error(int* err, int code) {

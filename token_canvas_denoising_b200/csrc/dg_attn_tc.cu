@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tile_src(i, mk, mv, y);
         uint8_t* kb = smem + kOffK + (i % kSlots) * kMatBytes;
         mbar_arrive_expect_tx(&k_full[i % kSlots], kMatBytes);
-        for (int a = 0; a < 2; ++a) tma_load_2d(kb + a * kAtom, mk, &k_full[i % kSlots], g * 128 + a * 64, y, pol);
+        tma_load_3d(kb, mk, &k_full[i % kSlots], 0, y, g * 2, pol);
       };
       auto load_v = [&](int i) {
         const CUtensorMap *mk, *mv;
@@ -181,15 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tile_src(i, mk, mv, y);
         uint8_t* vb = smem + kOffV + (i % kSlots) * kMatBytes;
         mbar_arrive_expect_tx(&v_full[i % kSlots], kMatBytes);
-        for (int a = 0; a < 2; ++a) tma_load_2d(vb + a * kAtom, mv, &v_full[i % kSlots], g * 128 + a * 64, y, pol);
+        tma_load_3d(vb, mv, &v_full[i % kSlots], 0, y, g * 2, pol);
       };
       // prompt-prefix tiles further ahead are pulled into L2 early
       auto prefetch = [&](int i) {
         if (i < n && t0 + i < nps) {
-          for (int a = 0; a < 2; ++a) {
-            tma_prefetch_2d(&maps.pk[lb], g * 128 + a * 64, (t0 + i) * kTile);
-            tma_prefetch_2d(&maps.pv[lb], g * 128 + a * 64, (t0 + i) * kTile);
-          }
+          tma_prefetch_3d(&maps.pk[lb], 0, (t0 + i) * kTile, g * 2);
+          tma_prefetch_3d(&maps.pv[lb], 0, (t0 + i) * kTile, g * 2);
         }
       };
       int nk = 0, nv = 0;  // next K tile and next V tile to load
@@ -204,8 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int i = nk; i < nk + kAhead; ++i) prefetch(i);
       griddep_wait();
       mbar_arrive_expect_tx(q_full, kMatBytes);
-      for (int a = 0; a < 2; ++a)
-        tma_load_2d(smem + kOffQ + a * kAtom, &maps.q, q_full, qh * 128 + a * 64, b * p.C + qt * kTile, pol);
+      tma_load_3d(smem + kOffQ, &maps.q, q_full, 0, b * p.C + qt * kTile, qh * 2, pol);
       // K runs one tile ahead of V
       while (nv < n && !*abort_flag) {
         if (nk < n && nk <= nv + 1) {
@@ -486,10 +483,12 @@ bool attn_tc_prepare(AttnTc* at, const AttnShape& sh, const void* Q, const void*
   at->part_ml = part_ml;
   at->splits = splits;
   at->groups.clear();
+  // [rows][heads * 128] bf16 as 3D (64 elements, rows, heads * 2): one box
+  // (64, 128, 2) is a head's 128 x 128 tile as two 128-byte-swizzled halves
   const uint64_t rows = (uint64_t)sh.B * sh.C;
-  const uint64_t dq[2] = {(uint64_t)sh.Hq * 128, rows}, sq[1] = {(uint64_t)sh.Hq * 256};
-  const uint64_t dk[2] = {(uint64_t)sh.Hk * 128, rows}, sk[1] = {(uint64_t)sh.Hk * 256};
-  const uint32_t box[2] = {64, 128};
+  const uint64_t dq[3] = {64, rows, (uint64_t)sh.Hq * 2}, sq[2] = {(uint64_t)sh.Hq * 256, 128};
+  const uint64_t dk[3] = {64, rows, (uint64_t)sh.Hk * 2}, sk[2] = {(uint64_t)sh.Hk * 256, 128};
+  const uint32_t box[3] = {64, 128, 2};
   for (int b0 = 0; b0 < sh.B; b0 += attntc::kMaxReq) {
     AttnTc::Group grp;
     grp.b0 = b0;
@@ -497,16 +496,16 @@ bool attn_tc_prepare(AttnTc* at, const AttnShape& sh, const void* Q, const void*
     static_assert(sizeof(attntc::Maps) <= sizeof(grp.maps), "AttnTc map storage too small");
     attntc::Maps* m = reinterpret_cast<attntc::Maps*>(grp.maps);
     memset(grp.maps, 0, sizeof(grp.maps));
-    if (!encode_tmap_bf16(&m->q, Q, 2, dq, sq, box, true) || !encode_tmap_bf16(&m->kc, Kc, 2, dk, sk, box, true) ||
-        !encode_tmap_bf16(&m->vc, Vc, 2, dk, sk, box, true))
+    if (!encode_tmap_bf16(&m->q, Q, 3, dq, sq, box, true) || !encode_tmap_bf16(&m->kc, Kc, 3, dk, sk, box, true) ||
+        !encode_tmap_bf16(&m->vc, Vc, 3, dk, sk, box, true))
       return false;
     for (int i = 0; i < grp.nreq; ++i) {
       const int b = b0 + i;
       grp.S[i] = S[b];
       if (S[b] > 0) {
-        const uint64_t dp[2] = {(uint64_t)sh.Hk * 128, (uint64_t)S[b]};
-        if (!encode_tmap_bf16(&m->pk[i], pk[b], 2, dp, sk, box, true) ||
-            !encode_tmap_bf16(&m->pv[i], pv[b], 2, dp, sk, box, true))
+        const uint64_t dp[3] = {64, (uint64_t)S[b], (uint64_t)sh.Hk * 2};
+        if (!encode_tmap_bf16(&m->pk[i], pk[b], 3, dp, sk, box, true) ||
+            !encode_tmap_bf16(&m->pv[i], pv[b], 3, dp, sk, box, true))
           return false;
       }
     }

@@ -10,7 +10,10 @@
 // while giving 2 CTAs per column tile for a 256-row canvas. The column tile is
 // chosen so that about one CTA per SM is launched; K is split only when even
 // 32-column tiles leave SMs idle. K-loop of 64-wide blocks through a TMA ring
-// of ~200 KB. Warp 0 issues TMA, warp 1 allocates TMEM and issues the MMAs
+// of ~200 KB; a stage holds KB consecutive K blocks of A and of W, each
+// fetched by one 3D box (64 elements, rows, K blocks): a TMA stream is bounded
+// by its per-box cost, so boxes are as large as the ring allows (KB = 4 for
+// BN <= 64, 2 for 128, 1 for 256). Warp 0 issues TMA, warp 1 allocates TMEM and issues the MMAs
 // (M=128, N=BN, K=16), warps 2..5 drain TMEM (warp w reads lanes 32*(w%4)).
 // With one split they add the residual, round and store; with several, every
 // CTA writes its f32 partial and a reduction kernel sums the partials in split
@@ -30,11 +33,16 @@ constexpr int kBM = 128;                        // rows per CTA
 constexpr int kABytes = kBM * 128;              // 16 KB per 64-wide K block
 constexpr int kThreads = 192;                   // TMA warp, MMA warp, 4 epilogue warps
 
+__host__ __device__ constexpr int kblocks_per_stage(int bn) { return bn <= 64 ? 4 : (bn == 128 ? 2 : 1); }
+
 template <int BN> struct Cfg {
-  static constexpr int kBBytes = BN * 128;
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kKB = kblocks_per_stage(BN);   // K blocks per stage (one box each for A and W)
+  static constexpr int kBBytes = BN * 128;            // W bytes per K block
+  static constexpr int kStageABytes = kKB * kABytes;
+  static constexpr int kStageBytes = kKB * (kABytes + kBBytes);
   static constexpr int kStages = (200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+  static_assert(kStages >= 2, "GEMM ring needs two stages");
 };
 
 struct Seg {
@@ -202,32 +210,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (lane == 0) {
       const uint64_t polA = policy_evict_last();
       const uint64_t polB = policy_evict_first();
-      const uint32_t bytes = kABytes + C::kBBytes;  // A rows past M are zero-filled
+      const uint32_t bytes = C::kStageBytes;  // rows past M / N and K blocks past K are zero-filled
       int s = 0;
       uint32_t ph = 0;
       bool issued[C::kStages];
       uint32_t issued_ph[C::kStages];
       for (int i = 0; i < C::kStages; ++i) issued[i] = false, issued_ph[i] = 0;
-      // weights are read-only inputs: the first stages' W tiles are fetched
+      // Stage u covers K blocks [kb0 + u KB, kb0 + (u + 1) KB) of this split.
+      // Every CTA walks K in the same order: the CTAs that share an A tile
+      // then request the same lines at about the same time, which L2 serves
+      // far faster than as many distinct lines.
+      const int nst = (kb1 - kb0 + C::kKB - 1) / C::kKB;
+      auto kstart = [&](int u) { return kb0 + u * C::kKB; };
+      // weights are read-only inputs: the first stages' W boxes are fetched
       // before waiting for the kernel that produces A
-      const int pre = min(C::kStages, kb1 - kb0);
+      const int pre = min(C::kStages, nst);
       for (int i = 0; i < pre; ++i) {
         uint8_t* st = smem + i * C::kStageBytes;
         mbar_arrive_expect_tx(&full[i], bytes);
-        tma_load_2d(st + kABytes, mapB, &full[i], (kb0 + i) * kBK, n0, polB);
+        tma_load_3d(st + C::kStageABytes, mapB, &full[i], 0, n0, kstart(i), polB);
         issued[i] = true;
         issued_ph[i] = 0;
       }
       griddep_wait();
-      for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * C::kStageBytes, &maps.a, &full[i], (kb0 + i) * kBK, m0, polA);
+      for (int i = 0; i < pre; ++i) tma_load_3d(smem + i * C::kStageBytes, &maps.a, &full[i], 0, m0, kstart(i), polA);
       s = pre % C::kStages;
       ph = (pre == C::kStages) ? 1u : 0u;
-      for (int kb = kb0 + pre; kb < kb1; ++kb) {
+      for (int u = pre; u < nst; ++u) {
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
         uint8_t* st = smem + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full[s], bytes);
-        tma_load_2d(st, &maps.a, &full[s], kb * kBK, m0, polA);
-        tma_load_2d(st + kABytes, mapB, &full[s], kb * kBK, n0, polB);
+        tma_load_3d(st, &maps.a, &full[s], 0, m0, kstart(u), polA);
+        tma_load_3d(st + C::kStageABytes, mapB, &full[s], 0, n0, kstart(u), polB);
         issued[s] = true;
         issued_ph[s] = ph;
         if (++s == C::kStages) { s = 0; ph ^= 1u; }
@@ -239,17 +253,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, BN);
+      const int nst = (kb1 - kb0 + C::kKB - 1) / C::kKB;
       int s = 0;
       uint32_t ph = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int u = 0; u < nst; ++u) {
+        // the same stage order as the producer; only the split's K blocks count
+        const int ks = kb0 + u * C::kKB;
+        const int nvalid = min(C::kKB, kb1 - ks);
         if (!mbar_wait(&full[s], ph, p.err, abort_flag)) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(smem + s * C::kStageBytes);
-        const uint32_t b0 = a0 + kABytes;
+        const uint32_t b0 = a0 + C::kStageABytes;
+        for (int j = 0; j < nvalid; ++j) {
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)
-          mma_bf16_ss(tmem, umma_desc_sw128(a0 + k * 32, 16, 1024), umma_desc_sw128(b0 + k * 32, 16, 1024), idesc,
-                      (kb > kb0 || k != 0) ? 1u : 0u);
+          for (int k = 0; k < kBK / 16; ++k)
+            mma_bf16_ss(tmem, umma_desc_sw128(a0 + j * kABytes + k * 32, 16, 1024),
+                        umma_desc_sw128(b0 + j * C::kBBytes + k * 32, 16, 1024), idesc,
+                        (u > 0 || j > 0 || k != 0) ? 1u : 0u);
+        }
         mma_commit(&empty[s]);
         if (++s == C::kStages) { s = 0; ph ^= 1u; }
       }
@@ -338,19 +359,22 @@ bool gemm_tc_prepare_with(GemmTc* g, const void* A, int M, int K, int nseg, cons
     return false;
   }
   g->bn = bn;
-  const uint64_t dA[2] = {(uint64_t)K, (uint64_t)M};
-  const uint64_t sA[1] = {(uint64_t)K * 2};
-  const uint32_t bA[2] = {64, (uint32_t)gemmtc::kBM};
-  if (!encode_tmap_bf16(&maps->a, A, 2, dA, sA, bA, true)) return false;
+  // K-major operands as 3D (64 elements, rows, K / 64) so that one box holds
+  // KB consecutive 128-byte-swizzled K blocks
+  const uint32_t kb = (uint32_t)gemmtc::kblocks_per_stage(bn);
+  const uint64_t dA[3] = {64, (uint64_t)M, (uint64_t)K / 64};
+  const uint64_t sA[2] = {(uint64_t)K * 2, 128};
+  const uint32_t bA[3] = {64, (uint32_t)gemmtc::kBM, kb};
+  if (!encode_tmap_bf16(&maps->a, A, 3, dA, sA, bA, true)) return false;
   g->M = M;
   g->K = K;
   g->nseg = nseg;
   g->tiles = 0;
   g->ncols = ncols;
   for (int i = 0; i < nseg; ++i) {
-    const uint64_t dB[2] = {(uint64_t)K, (uint64_t)N[i]};
-    const uint32_t bB[2] = {64, (uint32_t)g->bn};
-    if (!encode_tmap_bf16(&maps->b[i], W[i], 2, dB, sA, bB, true)) return false;
+    const uint64_t dB[3] = {64, (uint64_t)N[i], (uint64_t)K / 64};
+    const uint32_t bB[3] = {64, (uint32_t)g->bn, kb};
+    if (!encode_tmap_bf16(&maps->b[i], W[i], 3, dB, sA, bB, true)) return false;
     g->out[i] = out[i];
     g->N[i] = N[i];
     g->tiles += N[i] / g->bn;

@@ -139,6 +139,7 @@ struct MoeTc {
   void* hs_out = nullptr;    // residual stream out [M][d]
   float* logits = nullptr;   // [M][E]
   float* gate = nullptr;     // [M][topk]
+  int* sel = nullptr;        // [M][topk] chosen experts
   int* pos = nullptr;        // [M][topk + nsh]
   int* off = nullptr;        // [E + nsh + 1]
   int* pair_tok = nullptr;   // [R]

@@ -10,8 +10,10 @@
 //
 // Work split: CTA (p, mb) owns rows [256 mb, 256 mb + 256) and a contiguous run
 // of 32-column vocab granules; it walks that run in tiles of up to 256 columns.
-// Per tile: K-loop of 64-wide blocks, each a TMA load of the rows' A block (two
-// 128-row halves) and the tile's W rows, then 2 x 4 MMAs (M=128, N<=256, K=16)
+// Per tile: K-loop of 64-wide blocks, each two 256-row TMA boxes (the rows' A
+// block and 256 W rows from the tile's first granule; per-box cost, not bytes,
+// bounds a TMA stream, so boxes are as large as they go), then 2 x 4 MMAs
+// (M=128, N<=256, K=16)
 // into two TMEM accumulators (columns [0,256) and [256,512)). Eight epilogue
 // warps then stream the accumulators out of TMEM and fold them into each row's
 // online (max, Z, S, best, id) state in base 2 (exp2 on the MUFU). One
@@ -33,7 +35,7 @@ constexpr int kStages = 3;
 constexpr int kBK = 64;                        // bf16 per 128-byte row
 constexpr int kHalfBytes = 128 * 128;          // 128 rows x 128 B
 constexpr int kABytes = 2 * kHalfBytes;        // 32 KB
-constexpr int kGranule = 32;                   // vocab rows per B box
+constexpr int kGranule = 32;                   // vocab columns per work granule
 constexpr int kGranBytes = kGranule * 128;     // 4 KB
 constexpr int kMaxGran = 8;                    // 256-column tile
 constexpr int kBBytes = kMaxGran * kGranBytes; // 32 KB
@@ -113,36 +115,31 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       // vocab weights are read-only inputs: the first stages' W tiles are
       // fetched before waiting for the kernel that produces Hs
       int pre = 0;
+      // every stage is one 256-row A box and one 256-row W box (rows past M
+      // or V are zero-filled and still counted; unused rows are never read)
+      const uint32_t bytes = kStageBytes;
       if (n_tiles > 0) {
-        const int ng0 = min(kMaxGran, g1 - g0);
-        const uint32_t bytes0 = halves * kHalfBytes + ng0 * kGranBytes;
         pre = min(kStages, nk);
         for (int i = 0; i < pre; ++i) {
           uint8_t* st = smem + i * kStageBytes;
-          mbar_arrive_expect_tx(&full[i], bytes0);
-          for (int g = 0; g < ng0; ++g)
-            tma_load_2d(st + kABytes + g * kGranBytes, &tmB, &full[i], i * kBK, (g0 + g) * kGranule, polB);
+          mbar_arrive_expect_tx(&full[i], bytes);
+          tma_load_2d(st + kABytes, &tmB, &full[i], i * kBK, g0 * kGranule, polB);
           issued[i] = true;
           issued_ph[i] = 0;
         }
         griddep_wait();
-        for (int i = 0; i < pre; ++i)
-          for (int h = 0; h < halves; ++h)
-            tma_load_2d(smem + i * kStageBytes + h * kHalfBytes, &tmA, &full[i], i * kBK, m0 + h * 128, polA);
+        for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * kStageBytes, &tmA, &full[i], i * kBK, m0, polA);
         s = pre % kStages;
         ph = (pre == kStages) ? 1u : 0u;
       }
       for (int t = 0; t < n_tiles && !*abort_flag; ++t) {
         const int gt = g0 + t * kMaxGran;
-        const int ng = min(kMaxGran, g1 - gt);
-        const uint32_t bytes = halves * kHalfBytes + ng * kGranBytes;
         for (int kb = (t == 0 ? pre : 0); kb < nk; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
           uint8_t* st = smem + s * kStageBytes;
           mbar_arrive_expect_tx(&full[s], bytes);
-          for (int h = 0; h < halves; ++h) tma_load_2d(st + h * kHalfBytes, &tmA, &full[s], kb * kBK, m0 + h * 128, polA);
-          for (int g = 0; g < ng; ++g)
-            tma_load_2d(st + kABytes + g * kGranBytes, &tmB, &full[s], kb * kBK, (gt + g) * kGranule, polB);
+          tma_load_2d(st, &tmA, &full[s], kb * kBK, m0, polA);
+          tma_load_2d(st + kABytes, &tmB, &full[s], kb * kBK, gt * kGranule, polB);
           issued[s] = true;
           issued_ph[s] = ph;
           if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -295,9 +292,9 @@ bool lmhead_tc_prepare(const void* hs, const void* lm_head, int M, int d, int V,
   }
   const uint64_t dA[2] = {(uint64_t)d, (uint64_t)M};
   const uint64_t sA[1] = {(uint64_t)d * 2};
-  const uint32_t bA[2] = {64, 128};
+  const uint32_t bA[2] = {64, 256};
   const uint64_t dB[2] = {(uint64_t)d, (uint64_t)V};
-  const uint32_t bB[2] = {64, (uint32_t)lmtc::kGranule};
+  const uint32_t bB[2] = {64, (uint32_t)(lmtc::kMaxGran * lmtc::kGranule)};
   return encode_tmap_bf16(tmA, hs, 2, dA, sA, bA, true) && encode_tmap_bf16(tmB, lm_head, 2, dB, sA, bB, true);
 }
 

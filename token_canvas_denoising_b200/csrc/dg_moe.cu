@@ -4,8 +4,9 @@
 // 架构解剖 3: 128 fine-grained experts plus one shared expert, top-8 routing).
 //
 //   router   r = Hs Wr^T (f32)                      projection GEMM, f32 output
-//   route    p = softmax(r); top-k by p (lower expert id on ties); gates
-//            g = p_sel / sum p_sel; rows of each expert listed in token order
+//   top-k    p = softmax(r); top-k by p (lower expert id on ties); gates
+//            g = p_sel / sum p_sel (one warp per token)
+//   group    rows of each expert listed in token order (one block)
 //   gather   Xg[row] = Hs[token(row)]  (rows grouped by expert; shared experts
 //            take every token)
 //   gate/up  a = GELU(Xg W_gate^T) * (Xg W_up^T), rounded to bf16
@@ -35,93 +36,114 @@ struct RouteParams {
   const float* logits;  // [M][E]
   int M, E, topk, nsh;
   float* gate;          // [M][topk]
+  int* sel;             // [M][topk] chosen expert per (token, slot)
   int* pos;             // [M][topk + nsh] row of each (token, slot) in the grouped buffers
   int* off;             // [E + nsh + 1] first row of each expert (shared experts last)
   int* pair_tok;        // [M * (topk + nsh)] token of each grouped row
 };
 
-// One block of 1024 threads. Phase 1: one warp per token: softmax over the
-// E logits (E <= 256, 8 per lane), then top_k rounds of a warp argmax on
-// (probability, -expert id). Phase 2: row offsets per expert. Phase 3: one
-// warp per expert lists its tokens in token order (ballot + popc).
-__global__ void __launch_bounds__(1024) moe_route_kernel(RouteParams p) {
+// One warp per token: softmax over the E <= 256 router logits (8 per lane),
+// then top_k rounds of a warp argmax on (probability, -expert id); round k's
+// winner is kept by lane k, so the selection stays in registers.
+__global__ void __launch_bounds__(256) moe_topk_kernel(RouteParams p) {
+  griddep_launch();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= p.M) return;  // whole warp
+  float lv[8];
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    lv[j] = e < p.E ? p.logits[(size_t)t * p.E + e] : -INFINITY;
+    m = fmaxf(m, lv[j]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float ev[8], sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ev[j] = (lane + 32 * j < p.E) ? expf(lv[j] - m) : 0.f;
+    sum += ev[j];
+  }
+  sum = warp_sum(sum);
+  const float inv = 1.f / sum;
+  unsigned taken = 0u;
+  float my_p = 0.f;
+  int my_e = 0;
+#pragma unroll
+  for (int k = 0; k < kMaxTopK; ++k) {
+    if (k >= p.topk) break;  // uniform
+    float bv = -1.f;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      const float pv = ev[j] * inv;
+      if (!(taken >> j & 1u) && e < p.E && (pv > bv || (pv == bv && e < bi))) {
+        bv = pv;
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == k) {
+      my_p = bv;
+      my_e = bi;
+    }
+  }
+  const float psum = warp_sum(lane < p.topk ? my_p : 0.f);
+  if (lane < p.topk) {
+    p.gate[(size_t)t * p.topk + lane] = my_p / psum;
+    p.sel[(size_t)t * p.topk + lane] = my_e;
+  }
+}
+
+// One block of 1024 threads: per-expert counts, row offsets (shared experts
+// last), and for each expert its (token, slot) pairs in token order, one warp
+// per expert (ballot + popc over 32-token chunks).
+__global__ void __launch_bounds__(1024) moe_group_kernel(RouteParams p) {
   griddep_launch();
   griddep_wait();
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_off[kMaxE + 3];
-  __shared__ unsigned char s_sel[kMaxPairs];  // expert id per (token, slot)
+  __shared__ unsigned char s_sel[kMaxPairs];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int npairs = p.M * p.topk;
   for (int i = threadIdx.x; i < p.E; i += blockDim.x) s_cnt[i] = 0;
   __syncthreads();
-  for (int t = warp; t < p.M; t += nw) {
-    float lv[8];
-    float m = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane + 32 * j;
-      lv[j] = e < p.E ? p.logits[(size_t)t * p.E + e] : -INFINITY;
-      m = fmaxf(m, lv[j]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float ev[8], sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      ev[j] = (lane + 32 * j < p.E) ? expf(lv[j] - m) : 0.f;
-      sum += ev[j];
-    }
-    sum = warp_sum(sum);
-    const float inv = 1.f / sum;
-    unsigned taken = 0u;
-    float psel[kMaxTopK];
-    int esel[kMaxTopK];
-    float psum = 0.f;
-    for (int k = 0; k < p.topk; ++k) {
-      float bv = -1.f;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        const float pv = ev[j] * inv;
-        if (!(taken >> j & 1u) && e < p.E && (pv > bv || (pv == bv && e < bi))) {
-          bv = pv;
-          bi = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      psel[k] = bv;
-      esel[k] = bi;
-      psum += bv;
-    }
-    if (lane == 0) {
-      for (int k = 0; k < p.topk; ++k) {
-        p.gate[(size_t)t * p.topk + k] = psel[k] / psum;
-        s_sel[t * p.topk + k] = (unsigned char)esel[k];
-        atomicAdd(&s_cnt[esel[k]], 1);
-      }
-    }
+  for (int i = threadIdx.x; i < npairs; i += blockDim.x) {
+    const int e = p.sel[i];
+    s_sel[i] = (unsigned char)e;
+    atomicAdd(&s_cnt[e], 1);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int e = 0; e < p.E; ++e) {
-      s_off[e] = acc;
-      acc += s_cnt[e];
+  if (warp == 0) {  // exclusive prefix over the experts, 32 at a time
+    int base = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int c = (e0 + lane < p.E) ? s_cnt[e0 + lane] : 0;
+      int x = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (e0 + lane < p.E) s_off[e0 + lane] = base + x - c;
+      base += __shfl_sync(0xffffffffu, x, 31);
     }
-    for (int sh = 0; sh < p.nsh; ++sh) {
-      s_off[p.E + sh] = acc;
-      acc += p.M;
+    if (lane == 0) {
+      for (int sh = 0; sh < p.nsh; ++sh) s_off[p.E + sh] = base + sh * p.M;
+      s_off[p.E + p.nsh] = base + p.nsh * p.M;
     }
-    s_off[p.E + p.nsh] = acc;
   }
   __syncthreads();
   for (int i = threadIdx.x; i <= p.E + p.nsh; i += blockDim.x) p.off[i] = s_off[i];
@@ -362,7 +384,8 @@ __global__ void moe_combine_kernel(const __nv_bfloat16* __restrict__ Hs, const f
 size_t moe_workspace_bytes(const MoeShape& s) {
   const size_t R = (size_t)s.M * (s.topk + s.nsh);
   auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
-  return al(sizeof(float) * s.M * s.E) + al(sizeof(float) * s.M * s.topk) + al(sizeof(int) * s.M * (s.topk + s.nsh)) +
+  return al(sizeof(float) * s.M * s.E) + al(sizeof(float) * s.M * s.topk) + al(sizeof(int) * s.M * s.topk) +
+         al(sizeof(int) * s.M * (s.topk + s.nsh)) +
          al(sizeof(int) * (s.E + s.nsh + 1)) + al(sizeof(int) * R) + al(2 * R * s.d) + al(2 * R * s.I) +
          al(4 * R * s.d) + 8 * 256;
 }
@@ -392,6 +415,7 @@ bool moe_prepare(MoeTc* mt, const MoeShape& s, const void* hs, void* hs_out, con
   };
   mt->logits = reinterpret_cast<float*>(take(sizeof(float) * s.M * s.E));
   mt->gate = reinterpret_cast<float*>(take(sizeof(float) * s.M * s.topk));
+  mt->sel = reinterpret_cast<int*>(take(sizeof(int) * s.M * s.topk));
   mt->pos = reinterpret_cast<int*>(take(sizeof(int) * s.M * (s.topk + s.nsh)));
   mt->off = reinterpret_cast<int*>(take(sizeof(int) * (s.E + s.nsh + 1)));
   mt->pair_tok = reinterpret_cast<int*>(take(sizeof(int) * R));
@@ -435,10 +459,12 @@ void launch_moe(Exec& ex, const MoeTc& mt) {
   rp.topk = s.topk;
   rp.nsh = s.nsh;
   rp.gate = mt.gate;
+  rp.sel = mt.sel;
   rp.pos = mt.pos;
   rp.off = mt.off;
   rp.pair_tok = mt.pair_tok;
-  launch_pdl(moe::moe_route_kernel, dim3(1), dim3(1024), 0, ex.stream, rp);
+  launch_pdl(moe::moe_topk_kernel, dim3(ceil_div(s.M, 8)), dim3(256), 0, ex.stream, rp);
+  launch_pdl(moe::moe_group_kernel, dim3(1), dim3(1024), 0, ex.stream, rp);
   const int R = s.M * (s.topk + s.nsh);
   launch_pdl(moe::moe_gather_kernel, dim3(R), dim3(128), 0, ex.stream, static_cast<const __nv_bfloat16*>(mt.hs),
              (const int*)mt.pair_tok, static_cast<__nv_bfloat16*>(mt.xg), s.d);
@@ -458,7 +484,7 @@ void launch_moe(Exec& ex, const MoeTc& mt) {
   launch_pdl(moe::moe_combine_kernel, dim3(s.M), dim3(256), 0, ex.stream, static_cast<const __nv_bfloat16*>(mt.hs),
              (const float*)mt.y, (const int*)mt.pos, (const float*)mt.gate, static_cast<__nv_bfloat16*>(mt.hs_out), s.d,
              s.topk, s.nsh);
-  ex.launches += 5;
+  ex.launches += 6;
 }
 
 }  // namespace dg

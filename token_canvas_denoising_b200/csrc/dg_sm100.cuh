@@ -101,6 +101,13 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, i
                : "memory");
 }
 
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // 2D tiled load (box size fixed in the tensor map) into this CTA's shared
 // memory; completion is counted on `bar` in bytes. x is the innermost
 // coordinate (elements; x * element size must be a multiple of 16 bytes).

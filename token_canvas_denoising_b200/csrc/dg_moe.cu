@@ -194,8 +194,8 @@ constexpr int kStages = 3;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 
 struct FfnMaps {
-  CUtensorMap a0;  // gate/up: W_gate [E+nsh][I][d]; down: W_down [E+nsh][d][I]   (3D)
-  CUtensorMap a1;  // gate/up: W_up
+  CUtensorMap a0;  // gate/up: W_gate [E+nsh][I][d] (box 128 rows); down: W_down [E+nsh][d][I] (box 256 rows)
+  CUtensorMap a1;  // gate/up: W_up (box 128 rows); unused by down
   CUtensorMap b;   // gate/up: Xg [R][d]; down: act [R][I]                          (2D, box 32 rows)
 };
 
@@ -210,8 +210,10 @@ struct FfnParams {
 
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
 
-// CTA (128-row weight tile rt, expert e). MODE 0: two accumulators (gate, up)
-// of 128 x N in TMEM, GeGLU epilogue to act; MODE 1: one accumulator, f32 y.
+// CTA (weight tile rt, expert e); two 128 x N accumulators in TMEM, fed per
+// K block by the same B (the expert's token rows). MODE 0: a 128-row tile of
+// W_gate and of W_up, GeGLU epilogue to act. MODE 1: a 256-row tile of W_down
+// (one box) as two 128-row halves, f32 y.
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_constant__ FfnMaps maps, FfnParams p) {
   griddep_launch();
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr uint32_t kCols = MODE == 0 ? 512 : 256;
+  constexpr uint32_t kCols = 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
     if (lane == 0) {
       const uint64_t polW = policy_evict_first();
       const uint64_t polX = policy_evict_last();
-      const uint32_t bytes = (MODE == 0 ? 2 : 1) * kATile + nbox * kBox * 128;
+      const uint32_t bytes = 2 * kATile + nbox * kBox * 128;
       int s = 0;
       uint32_t ph = 0;
       bool issued[kStages] = {false, false, false};
@@ -265,8 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
         uint8_t* st = smem + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], bytes);
-        tma_load_3d(st, &maps.a0, &full[s], kb * 64, rt * 128, e, polW);
-        if (MODE == 0) tma_load_3d(st + kATile, &maps.a1, &full[s], kb * 64, rt * 128, e, polW);
+        if (MODE == 0) {
+          tma_load_3d(st, &maps.a0, &full[s], kb * 64, rt * 128, e, polW);
+          tma_load_3d(st + kATile, &maps.a1, &full[s], kb * 64, rt * 128, e, polW);
+        } else {
+          tma_load_3d(st, &maps.a0, &full[s], kb * 64, rt * 256, e, polW);  // 256 rows = both halves
+        }
         for (int bx = 0; bx < nbox; ++bx)
           tma_load_2d(st + 2 * kATile + bx * kBox * 128, &maps.b, &full[s], kb * 64, r0 + bx * kBox, polX);
         issued[s] = true;
@@ -291,8 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
         for (int k = 0; k < 4; ++k) {
           const uint64_t bd = umma_desc_sw128(b0 + k * 32, 16, 1024);
           mma_bf16_ss(tmem, umma_desc_sw128(a0 + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
-          if (MODE == 0)
-            mma_bf16_ss(tmem + 256, umma_desc_sw128(a0 + kATile + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
+          mma_bf16_ss(tmem + 256, umma_desc_sw128(a0 + kATile + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
         }
         mma_commit(&empty[s]);
         if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -301,7 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
     }
   } else {
     const int quad = warp & 3;
-    const int row = rt * 128 + quad * 32 + lane;  // weight row: I index (MODE 0) or d index (MODE 1)
+    // weight row: I index (MODE 0) or d index of the first half (MODE 1)
+    const int row = rt * (MODE == 0 ? 128 : 256) + quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const bool ok = mbar_wait_warp(tfull, 0, p.err, abort_flag);
     tc_fence_after();
@@ -322,11 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
               }
             }
           }
-        } else if (row < p.rows) {
+        } else {
+          uint32_t g1[32];
+          tmem_ld32_sync(tmem + lane_off + 256 + c * 32, g1);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int tok = c * 32 + j;
-            if (tok < n) p.y[(size_t)(r0 + tok) * p.rows + row] = __uint_as_float(g[j]);
+            if (tok < n && row < p.rows) p.y[(size_t)(r0 + tok) * p.rows + row] = __uint_as_float(g[j]);
+            if (tok < n && row + 128 < p.rows) p.y[(size_t)(r0 + tok) * p.rows + row + 128] = __uint_as_float(g1[j]);
           }
         }
       }
@@ -439,12 +448,13 @@ bool moe_prepare(MoeTc* mt, const MoeShape& s, const void* hs, void* hs_out, con
   const uint64_t ddn[3] = {(uint64_t)s.I, (uint64_t)s.d, ne_tot};
   const uint64_t sdn[2] = {(uint64_t)s.I * 2, (uint64_t)s.d * s.I * 2};
   const uint32_t bw[3] = {64, 128, 1};
+  const uint32_t bw_dn[3] = {64, 256, 1};
   const uint64_t dx[2] = {(uint64_t)s.d, R}, sx[1] = {(uint64_t)s.d * 2};
   const uint64_t da[2] = {(uint64_t)s.I, R}, sa[1] = {(uint64_t)s.I * 2};
   const uint32_t bb[2] = {64, (uint32_t)moe::kBox};
   if (!encode_tmap_bf16(&gu->a0, w_gate, 3, dgu, sgu, bw, true) || !encode_tmap_bf16(&gu->a1, w_up, 3, dgu, sgu, bw, true) ||
-      !encode_tmap_bf16(&gu->b, mt->xg, 2, dx, sx, bb, true) || !encode_tmap_bf16(&dn->a0, w_down, 3, ddn, sdn, bw, true) ||
-      !encode_tmap_bf16(&dn->a1, w_down, 3, ddn, sdn, bw, true) || !encode_tmap_bf16(&dn->b, mt->act, 2, da, sa, bb, true))
+      !encode_tmap_bf16(&gu->b, mt->xg, 2, dx, sx, bb, true) || !encode_tmap_bf16(&dn->a0, w_down, 3, ddn, sdn, bw_dn, true) ||
+      !encode_tmap_bf16(&dn->a1, w_down, 3, ddn, sdn, bw_dn, true) || !encode_tmap_bf16(&dn->b, mt->act, 2, da, sa, bb, true))
     return false;
   return true;
 }
@@ -479,7 +489,7 @@ void launch_moe(Exec& ex, const MoeTc& mt) {
              ex.stream, *reinterpret_cast<const moe::FfnMaps*>(mt.maps_gateup), fp);
   fp.K = s.I;
   fp.rows = s.d;
-  launch_pdl(moe::moe_ffn_kernel<1>, dim3(ceil_div(s.d, 128), s.E + s.nsh), dim3(moe::kThreads), moe::kSmemBytes,
+  launch_pdl(moe::moe_ffn_kernel<1>, dim3(ceil_div(s.d, 256), s.E + s.nsh), dim3(moe::kThreads), moe::kSmemBytes,
              ex.stream, *reinterpret_cast<const moe::FfnMaps*>(mt.maps_down), fp);
   launch_pdl(moe::moe_combine_kernel, dim3(s.M), dim3(256), 0, ex.stream, static_cast<const __nv_bfloat16*>(mt.hs),
              (const float*)mt.y, (const int*)mt.pos, (const float*)mt.gate, static_cast<__nv_bfloat16*>(mt.hs_out), s.d,

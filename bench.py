@@ -31,6 +31,31 @@ BLOCK_STEPS = 48
 REF_BUDGET_S = 150.0  # target wall time of the whole reference-arm run
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(value, world, device):
+    """The largest value over the ranks (a device time: the job is as slow as
+    its slowest rank). One all-reduce on `device` ('cuda' under NCCL, 'cpu'
+    under gloo); every rank calls it at the same point."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, elapsed_ms):
+    """Whole-job throughput: the units every rank processed / the slowest
+    rank's elapsed time."""
+    return world * units_per_rank / (elapsed_ms / 1e3)
+
+
+def rank_canvas_seeds(seeds, rank):
+    """Each rank decodes its own requests: canvas seeds offset per rank."""
+    return tuple(int(s) + 1000 * rank for s in seeds)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -228,7 +253,7 @@ def bench_b200(args, rank, world, local_rank):
 
     cfg = workload_cfg(args.workload)
     # each rank decodes its own requests: distinct canvas seeds per rank
-    cfg_r = fx.derive(cfg, canvas_seeds=tuple(s + 1000 * rank for s in cfg.canvas_seeds))
+    cfg_r = fx.derive(cfg, canvas_seeds=rank_canvas_seeds(cfg.canvas_seeds, rank))
     wl = fx.make_workload(cfg_r)
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
@@ -272,9 +297,7 @@ def bench_b200(args, rank, world, local_rank):
     cv.sync()
     n_resets = (args.steps - 1) // BLOCK_STEPS
     if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+        elapsed_ms = max_over_ranks(elapsed_ms, world, "cuda")
         dist.barrier()
 
     # ---- timed region 2: the same steps with CUDA events recorded around the
@@ -304,7 +327,7 @@ def bench_b200(args, rank, world, local_rank):
     for j in range(max(0, lm_steps - (NEV - 1)), lm_steps):
         lm_ms.append(ev_s[j % NEV].elapsed_time(ev_e[j % NEV]))
     cv.set_timing_events([], [])
-    steps_per_s = world * args.steps / (elapsed_ms / 1e3)
+    steps_per_s = job_rate(args.steps, world, elapsed_ms)
     lm_avg_ms = float(np.mean(lm_ms))
     lm_tflops = fb["flops_lm"] / (lm_avg_ms / 1e3) / 1e12
 
@@ -333,15 +356,13 @@ def bench_b200(args, rank, world, local_rank):
         e2e_ms = e0.elapsed_time(e1)
         h2d = sum(v.nbytes for v in pin_np.values())
         d2h = tok_out.numel() * 4 + cfg.B * 4
-        e2e = {"value": world * total_steps / (e2e_ms / 1e3), "unit": "steps/s",
+        e2e = {"value": job_rate(total_steps, world, e2e_ms), "unit": "steps/s",
                "h2d_bytes_per_step": int(round(h2d / BLOCK_STEPS)),
                "d2h_bytes_per_step": int(round(d2h / BLOCK_STEPS)),
                "note": f"{args.e2e_blocks} decode blocks of {BLOCK_STEPS} steps via dg_canvas_set_state "
                        "(pinned host -> device) + dg_decode_block (tokens to pinned host)"}
         if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e["value"] = world * total_steps / (float(t.item()) / 1e3)
+            e2e["value"] = job_rate(total_steps, world, max_over_ranks(e2e_ms, world, "cuda"))
 
     cpu = None
     if rank == 0 and world == 1:

@@ -23,7 +23,7 @@ What the pages fix, and where (page title, section):
   * MoE FFN: 128 fine-grained experts plus one shared expert, top-8 routing --
     "DiffusionGemma深度拆解" 架构解剖 3.
 
-Readings where the pages are silent (listed in the design doc as well): single
+Readings where the pages are silent: single
 layer, embed -> attention -> Wo + residual (-> MoE + residual) -> LM head, no
 norm and no positional encoding; KV head g = q // (Hq/Hk); softmax scale
 1/sqrt(h); freeze count k_t = ceil(U_t / (T - t)); freeze set = the k_t

@@ -78,7 +78,16 @@ typedef struct dg_model_desc {
   const void *wv;       /* [n_kv_heads*head_dim][d_model]         */
   const void *wo;       /* [d_model][n_q_heads*head_dim]          */
   const void *lm_head;  /* [vocab][d_model]                       */
-  /* MoE FFN after attention; n_experts = 0 disables it. */
+  /* MoE FFN after attention ([P3] 架构解剖 3); n_experts = 0 disables it.
+   * r = Hs W_router^T; p = softmax(r); the top_k experts by p (lower expert id
+   * on ties) with gates g = p / sum of the chosen p; for each chosen and each
+   * shared expert e: FFN_e(x) = W_down[e] (GELU(W_gate[e] x) * (W_up[e] x))
+   * (exact-erf GELU, the product rounded to the storage dtype); Hs becomes
+   * Hs + sum g_e FFN_e(Hs) + sum_shared FFN_e(Hs), rounded to the storage
+   * dtype. Shared experts are stored after the routed ones. Supported (else
+   * DG_ERR_UNSUPPORTED): bf16 only, n_experts a multiple of 32 and <= 256,
+   * top_k <= 8, n_shared <= 2, moe_inter a multiple of 64, batch * canvas_len
+   * <= 256. */
   int32_t n_experts, top_k, moe_inter, n_shared;
   const void *w_router; /* [n_experts][d_model]                   */
   const void *w_gate;   /* [n_experts+n_shared][moe_inter][d_model] */

@@ -158,6 +158,21 @@ dg_status dg_denoise_step(dg_ctx *ctx, const dg_schedule *sched, const dg_step_o
  * keeps the current seeds), clear the frozen and done flags. Asynchronous. */
 dg_status dg_canvas_reset(dg_ctx *ctx, const uint64_t *seeds);
 
+/* Start a new block with some positions given in advance: infilling between a
+ * given prefix and suffix, or a puzzle's given cells ([P3] 为什么值得重视 2:
+ * fill-in-the-middle, constraints propagating from every direction; [P4]
+ * 工作原理: constrained generation). As dg_canvas_reset, then every position
+ * with fixed_mask[i] != 0 takes fixed_tokens[i] and starts frozen: it keeps
+ * its token, keeps contributing K/V, and the freeze schedule counts only the
+ * open positions (k_t = ceil(U_t / (T - t)) over the unfrozen ones).
+ *   seeds         host [B] or NULL (keep the current seeds).
+ *   fixed_mask    host [B*C] uint8 (canvas-major), nonzero = given.
+ *   fixed_tokens  host [B*C] int32; read only where fixed_mask is set, each
+ *                 in [0, vocab) (else DG_ERR_INVALID_ARG before any work).
+ * Synchronous. A canvas whose positions are all given stops after one step. */
+dg_status dg_canvas_reset_fixed(dg_ctx *ctx, const uint64_t *seeds, const uint8_t *fixed_mask,
+                                const int32_t *fixed_tokens);
+
 /* Denoise until every canvas is done (at most sched->max_steps steps each).
  *   tokens_out  [B*C] int32, device or host memory (copied with UVA), or NULL.
  *   steps_out   host [B] steps taken per canvas, or NULL.

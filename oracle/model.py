@@ -251,6 +251,22 @@ def init_state(seeds, C, V):
     }
 
 
+def init_state_fixed(seeds, C, V, fixed_mask, fixed_tok):
+    """A block with some positions given in advance: infilling between a given
+    prefix and suffix, or a puzzle's given cells ("DiffusionGemma深度拆解" 为什么值得
+    重视 2, fill-in-the-middle, constraints propagating from every direction;
+    "谷歌DiffusionGemma" 工作原理, constrained generation). Positions with
+    fixed_mask take fixed_tok and start frozen, so they keep their tokens and
+    only the open positions count as unfrozen in the freeze schedule; every
+    other position starts at its step-0 draw, as in init_state."""
+    st = init_state(seeds, C, V)
+    mask = np.asarray(fixed_mask, dtype=bool).reshape(st["tok"].shape)
+    tok = np.asarray(fixed_tok, dtype=np.int64).reshape(st["tok"].shape)
+    st["tok"] = np.where(mask, tok, st["tok"])
+    st["frozen"] = mask.copy()
+    return st
+
+
 def copy_state(st):
     return {k: v.copy() for k, v in st.items()}
 

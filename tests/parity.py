@@ -254,13 +254,13 @@ def lm_column_absmax(omodel):
 
 
 def run_lockstep(cfg, canvas, omodel, oprefix, osched, abi_sched, inv_temp, n_steps=None,
-                 free_running=True, check_tensors=True):
+                 free_running=True, check_tensors=True, init=None):
     """Drive GPU and oracle side by side. In free-running mode the GPU keeps its
     own state while no ambiguous decision has happened; after one, and always in
     lock-step mode, the GPU restarts each step from the oracle's state.
     Returns the StepReport."""
     rep = StepReport()
-    ost = om.init_state(np.array(cfg.canvas_seeds, dtype=np.uint64), cfg.C, cfg.V)
+    ost = om.init_state(np.array(cfg.canvas_seeds, dtype=np.uint64), cfg.C, cfg.V) if init is None else init
     g0 = canvas.get_state()
     init = abi_state_to_oracle(g0, cfg.B, cfg.C)
     if not np.array_equal(init["tok"], ost["tok"]):

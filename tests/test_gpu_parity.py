@@ -82,6 +82,38 @@ def test_bf16_moe_uneven_experts():
     _run(cfg, n_steps=3)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fixed_positions_full_decode(dtype):
+    """Infilling: a given prefix and suffix of each canvas (and one given cell
+    in the middle of the second) stay fixed while the rest is decoded; full
+    decode against the oracle started from the same given positions."""
+    from token_canvas_denoising_b200.canvas import schedule
+    if dtype == "f32":
+        cfg = fx.Config("fixed_f32", B=2, C=24, S=(10, 33), d=64, Hq=2, Hk=1, h=32, V=300, dtype="f32",
+                        max_steps=7, weight_seed=3, canvas_seeds=(1, 2))
+    else:
+        cfg = fx.Config("fixed_bf16", B=2, C=130, S=(100, 40), d=128, Hq=2, Hk=1, h=128, V=1024,
+                        dtype="bf16", max_steps=12, weight_seed=31, canvas_seeds=(4, 5))
+    wl = fx.make_workload(cfg)
+    mask = np.zeros((cfg.B, cfg.C), bool)
+    mask[:, :cfg.C // 5] = True
+    mask[:, cfg.C - cfg.C // 6:] = True
+    mask[1, cfg.C // 2] = True
+    toks = np.random.default_rng(7).integers(0, cfg.V, size=(cfg.B, cfg.C))
+    cv, keep = _canvas(wl)
+    try:
+        cv.reset(fixed_mask=mask, fixed_tokens=toks)
+        ost = om.init_state_fixed(wl.seeds, cfg.C, cfg.V, mask, toks)
+        rep, steps = run_lockstep(cfg, cv, oracle_model(wl), oracle_prefix(wl), oracle_sched(cfg, adaptive=True),
+                                  schedule(cfg.max_steps, cfg.stop_entropy, True), None, init=ost)
+        final = cv.get_state()
+    finally:
+        cv.close()
+    assert not rep.errors, "\n".join(rep.errors[:20])
+    assert np.array_equal(final["tokens"].reshape(cfg.B, cfg.C)[mask], toks[mask])
+    assert np.all(final["done"])
+
+
 def test_decode_block_matches_stepping():
     """dg_decode_block (device loop) ends in the same state as single steps."""
     from token_canvas_denoising_b200.canvas import from_workload, schedule

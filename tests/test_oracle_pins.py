@@ -337,6 +337,61 @@ def test_adaptive_stop_uses_threshold():
     assert len(recs) == 1 and np.all(final["tok"] == 5)
 
 
+# ---------------------------------------------------------------- fixed positions
+def test_fixed_positions_empty_mask_is_the_plain_block():
+    cfg = _tiny_loop_cfg(V=8, C=6)
+    wl = fx.make_workload(cfg)
+    a = oracle_init(wl)
+    b = om.init_state_fixed(wl.seeds, cfg.C, cfg.V, np.zeros((1, cfg.C), bool), np.zeros((1, cfg.C), int))
+    assert np.array_equal(a["tok"], b["tok"]) and not b["frozen"].any()
+
+
+def test_fixed_positions_keep_tokens_and_only_open_positions_are_scheduled():
+    """C = 16, T = 8, 6 positions given: the schedule runs over the 10 open ones,
+    k_t = ceil(U / (T - t)) with U = 10, 8, 6, 5, 4, 3, 2, 1 (worked by hand)."""
+    cfg = fx.Config(name="fixed", B=1, C=16, S=(3,), d=8, Hq=2, Hk=1, h=4, V=8, dtype="f32",
+                    max_steps=8, weight_seed=11, canvas_seeds=(9,))
+    wl = fx.make_workload(cfg)
+    mask = np.zeros((1, 16), bool)
+    mask[0, [0, 1, 2, 13, 14, 15]] = True  # a given prefix and suffix; the middle is filled
+    given = np.zeros((1, 16), int)
+    given[0, [0, 1, 2, 13, 14, 15]] = [3, 1, 4, 1, 5, 7]
+    st0 = om.init_state_fixed(wl.seeds, cfg.C, cfg.V, mask, given)
+    final, recs = om.decode(oracle_model(wl), oracle_prefix(wl), st0, oracle_sched(cfg, False))
+    _check_trajectory(cfg, st0, final, recs, False)
+    assert [int(r["canvas"][0]["freeze"].sum()) for r in recs] == [2, 2, 1, 1, 1, 1, 1, 1]
+    assert np.array_equal(final["tok"][mask], given[mask])
+    # the open positions were drawn like any other block
+    for p in np.nonzero(~mask[0])[0]:
+        assert st0["tok"][0, p] == op.canvas_draw(int(cfg.canvas_seeds[0]), 0, int(p), 0, cfg.V)
+
+
+def test_all_positions_fixed_ends_after_one_step():
+    cfg = _tiny_loop_cfg(V=8, C=6)
+    wl = fx.make_workload(cfg)
+    given = np.array([[7, 6, 5, 4, 3, 2]])
+    st0 = om.init_state_fixed(wl.seeds, cfg.C, cfg.V, np.ones((1, cfg.C), bool), given)
+    final, recs = om.decode(oracle_model(wl), oracle_prefix(wl), st0, oracle_sched(cfg, False))
+    assert len(recs) == 1 and np.array_equal(final["tok"], given) and final["done"].all()
+
+
+@pytest.mark.parametrize("adaptive", [False, True])
+def test_one_fixed_position_all_canvases_v2_c4(adaptive):
+    """Every initial canvas of V = 2, C = 4 with position 1 given as either
+    token: the trajectory invariants hold and the given token survives."""
+    cfg = _tiny_loop_cfg()
+    wl = fx.make_workload(cfg)
+    m = oracle_model(wl)
+    sched = oracle_sched(cfg, adaptive=adaptive)
+    mask = np.array([[False, True, False, False]])
+    for init in itertools.product(range(cfg.V), repeat=cfg.C):
+        st0 = om.init_state_fixed(wl.seeds, cfg.C, cfg.V, mask, np.array([init]))
+        st0["tok"][0] = np.array(init)
+        final, recs = om.decode(m, oracle_prefix(wl), st0, sched)
+        _check_trajectory(cfg, st0, final, recs, adaptive)
+        assert final["tok"][0, 1] == init[1]
+
+
 # ---------------------------------------------------------------- MoE
 def _moe_cfg():
     return fx.Config(name="moe_t", B=1, C=5, S=(3,), d=12, Hq=2, Hk=1, h=4, V=16, dtype="f32",

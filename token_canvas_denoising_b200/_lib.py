@@ -52,6 +52,7 @@ SIGNATURES = {
     "dg_canvas_set_state": (C.c_int, [C.c_void_p, C.POINTER(dg_state)]),
     "dg_canvas_sync": (C.c_int, [C.c_void_p]),
     "dg_canvas_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "dg_canvas_reset_fixed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_canvas_set_timing_events": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]),
     "dg_canvas_destroy": (None, [C.c_void_p]),
     "dg_status_string": (C.c_char_p, [C.c_int]),

@@ -117,13 +117,26 @@ class DenoiseCanvas:
         hs = L.dg_state(*[arrs[k].ctypes.data for k in ("tokens", "frozen", "step", "seed", "done")])
         L.check(self._lib.dg_canvas_set_state(self._ctx, C.byref(hs)), "dg_canvas_set_state")
 
-    def reset(self, seeds=None):
-        """Redraw every canvas at step 0 (device side, asynchronous)."""
+    def reset(self, seeds=None, fixed_mask=None, fixed_tokens=None):
+        """Redraw every canvas at step 0 (device side, asynchronous). With
+        fixed_mask / fixed_tokens ([B][C] or [B*C] arrays), the given positions
+        take the given tokens and start frozen (synchronous)."""
         arr = None
         if seeds is not None:
             arr = (C.c_uint64 * self.B)(*[int(x) for x in seeds])
-        st = self._lib.dg_canvas_reset(self._ctx, C.cast(arr, C.c_void_p) if arr is not None else None)
-        L.check(st, "dg_canvas_reset")
+        seeds_p = C.cast(arr, C.c_void_p) if arr is not None else None
+        if fixed_mask is None:
+            st = self._lib.dg_canvas_reset(self._ctx, seeds_p)
+            L.check(st, "dg_canvas_reset")
+            return
+        import numpy as np
+        mask = np.ascontiguousarray(np.asarray(fixed_mask).reshape(-1) != 0, dtype=np.uint8)
+        toks = np.ascontiguousarray(np.asarray(fixed_tokens).reshape(-1), dtype=np.int32)
+        if mask.size != self.M or toks.size != self.M:
+            raise ValueError(f"fixed_mask and fixed_tokens need {self.M} entries")
+        st = self._lib.dg_canvas_reset_fixed(self._ctx, seeds_p, mask.ctypes.data_as(C.c_void_p),
+                                             toks.ctypes.data_as(C.c_void_p))
+        L.check(st, "dg_canvas_reset_fixed")
 
     def set_timing_events(self, starts, stops):
         """Record torch.cuda.Event pairs around the LM-head kernel of graph steps

@@ -438,6 +438,29 @@ dg_status dg_canvas_reset(dg_ctx* ctx, const uint64_t* seeds) {
   return check_launch("reset canvas");
 }
 
+dg_status dg_canvas_reset_fixed(dg_ctx* ctx, const uint64_t* seeds, const uint8_t* fixed_mask,
+                                const int32_t* fixed_tokens) {
+  DG_ARG(ctx != nullptr, "ctx is NULL");
+  DG_ARG(fixed_mask && fixed_tokens, "fixed_mask / fixed_tokens is NULL");
+  for (int i = 0; i < ctx->M; ++i)
+    if (fixed_mask[i]) DG_ARG(fixed_tokens[i] >= 0 && fixed_tokens[i] < ctx->m.vocab, "fixed token id out of range");
+  dg_status st = dg_canvas_reset(ctx, seeds);
+  if (st != DG_OK) return st;
+  // the step-0 draws of the open positions stay; the given ones overwrite theirs
+  std::vector<int32_t> tok(ctx->M);
+  std::vector<uint8_t> frozen(ctx->M);
+  DG_CUDA_RET(cudaMemcpyAsync(tok.data(), ctx->cs.tok, ctx->M * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
+  for (int i = 0; i < ctx->M; ++i) {
+    frozen[i] = fixed_mask[i] ? 1 : 0;
+    if (fixed_mask[i]) tok[i] = fixed_tokens[i];
+  }
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.tok, tok.data(), ctx->M * sizeof(int32_t), cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.frozen, frozen.data(), ctx->M, cudaMemcpyHostToDevice, ctx->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
+  return read_device_error(ctx);
+}
+
 dg_status dg_decode_block(dg_ctx* ctx, const dg_schedule* sched, int32_t* tokens_out, int32_t* steps_out) {
   DG_ARG(ctx != nullptr, "ctx is NULL");
   dg_status st = validate_sched(sched);

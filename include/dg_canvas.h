@@ -173,6 +173,29 @@ dg_status dg_canvas_reset(dg_ctx *ctx, const uint64_t *seeds);
 dg_status dg_canvas_reset_fixed(dg_ctx *ctx, const uint64_t *seeds, const uint8_t *fixed_mask,
                                 const int32_t *fixed_tokens);
 
+/* Block-autoregressive decoding: after a canvas is committed, its tokens'
+ * K/V join the request's cached prompt and the next canvas attends to both
+ * ([P3] 架构解剖 1: blocks in sequence, parallel within a block; the committed
+ * block's K/V come from the causal encoder pass). With one layer and no
+ * positional encoding a token's K/V depend only on its embedding, so the
+ * encoder pass is the K/V projection of the committed tokens.
+ *
+ * dg_canvas_block_kv writes the K/V of the current canvas tokens:
+ *   k_out, v_out  device [B*C][n_kv_heads*head_dim] in the storage dtype,
+ *                 canvas-major (rows b*C .. b*C+C-1 belong to request b), the
+ *                 same per-token layout as the prompt cache, so appending a
+ *                 request's rows to its cache is a plain copy.
+ * Asynchronous; overwrites the context's step scratch (call between steps). */
+dg_status dg_canvas_block_kv(dg_ctx *ctx, void *k_out, void *v_out);
+
+/* Point the context at new prompt K/V caches (e.g. the old prefix followed by
+ * a committed block): arguments as in dg_canvas_init (host [B] lengths,
+ * host arrays of device pointers, 16-byte aligned, caller-owned). Waits for the
+ * queued work; the next step re-captures its graph. The canvas state is not
+ * touched (use dg_canvas_reset to start the next block). */
+dg_status dg_canvas_set_prefix(dg_ctx *ctx, const int32_t *prefix_len, const void *const *prefix_k,
+                               const void *const *prefix_v);
+
 /* Denoise until every canvas is done (at most sched->max_steps steps each).
  *   tokens_out  [B*C] int32, device or host memory (copied with UVA), or NULL.
  *   steps_out   host [B] steps taken per canvas, or NULL.

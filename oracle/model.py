@@ -90,6 +90,32 @@ def project_qkv(model, X):
     return Q, Kc, Vc
 
 
+def block_kv(model, tok):
+    """K and V of committed canvases, as stored: the next block attends to them
+    after the request's prompt ("DiffusionGemma深度拆解" 架构解剖 1: blocks in
+    sequence, parallel inside a block; the committed block's K/V come from the
+    causal encoder pass). With one layer and no positional encoding a token's
+    K/V depend only on its own embedding, so that pass is the K/V projection of
+    the committed tokens. tok: [B][C]; returns K, V as [B][C][Hk][h] (fp64
+    values rounded to the storage dtype)."""
+    B, C = np.asarray(tok).shape
+    _, Kc, Vc = project_qkv(model, embed(model, tok))
+    _, _, Hk, h, _ = dims(model)
+    return Kc.reshape(B, C, Hk, h), Vc.reshape(B, C, Hk, h)
+
+
+def append_block(model, prefix, K, V):
+    """Each request's prompt K/V followed by its committed block's K/V (fp64)."""
+    _, _, Hk, h, _ = dims(model)
+    dt = model["dtype"]
+    out = []
+    for b, (pk, pv) in enumerate(prefix):
+        pk = widen(pk, dt).reshape(-1, Hk, h)
+        pv = widen(pv, dt).reshape(-1, Hk, h)
+        out.append((np.concatenate([pk, K[b]]), np.concatenate([pv, V[b]])))
+    return out
+
+
 def softmax_rows(s):
     m = np.max(s, axis=-1, keepdims=True)
     e = np.exp(s - m)

@@ -294,4 +294,5 @@ def run_lockstep(cfg, canvas, omodel, oprefix, osched, abi_sched, inv_temp, n_st
             synced = False
         ost = ost_next
         steps += 1
+    rep.final_state = ost
     return rep, steps

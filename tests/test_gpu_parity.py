@@ -114,6 +114,50 @@ def test_fixed_positions_full_decode(dtype):
     assert np.all(final["done"])
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_two_blocks_in_sequence(dtype):
+    """Block-autoregressive decoding: block 1 is decoded and committed, its K/V
+    (dg_canvas_block_kv, checked against the oracle) are appended to each
+    request's prompt cache (dg_canvas_set_prefix), and block 2 is decoded over
+    prompt + block 1 against the oracle doing the same."""
+    from token_canvas_denoising_b200.canvas import schedule
+    from tests.parity import close, oracle_state_to_abi
+    if dtype == "f32":
+        cfg = fx.Config("blocks_f32", B=2, C=24, S=(10, 33), d=64, Hq=2, Hk=1, h=32, V=300, dtype="f32",
+                        max_steps=7, weight_seed=3, canvas_seeds=(1, 2))
+    else:
+        cfg = fx.Config("blocks_bf16", B=2, C=130, S=(100, 0), d=128, Hq=2, Hk=1, h=128, V=1024,
+                        dtype="bf16", max_steps=8, weight_seed=37, canvas_seeds=(6, 7))
+    wl = fx.make_workload(cfg)
+    m, pre = oracle_model(wl), oracle_prefix(wl)
+    sched, osched = schedule(cfg.max_steps, cfg.stop_entropy, True), oracle_sched(cfg, adaptive=True)
+    cv, keep = _canvas(wl)
+    try:
+        rep1, _ = run_lockstep(cfg, cv, m, pre, osched, sched, None)
+        assert not rep1.errors, "\n".join(rep1.errors[:20])
+        ost = rep1.final_state
+        cv.set_state(oracle_state_to_abi(ost))  # both sides commit the same tokens
+        K, V = cv.block_kv()
+        Ko, Vo = om.block_kv(m, ost["tok"])
+        for g, o in ((K, Ko), (V, Vo)):
+            n, mx = close(g.float().cpu().numpy(), o.reshape(cfg.B * cfg.C, -1))
+            assert n == 0, f"block K/V: {n} elements out of tolerance (max abs diff {mx:.3g})"
+        kv = (cfg.Hk, cfg.h)
+        new_pk = [torch.cat([keep["prefix_k"][b].reshape(-1, *kv),
+                             K[b * cfg.C:(b + 1) * cfg.C].reshape(cfg.C, *kv)]).contiguous() for b in range(cfg.B)]
+        new_pv = [torch.cat([keep["prefix_v"][b].reshape(-1, *kv),
+                             V[b * cfg.C:(b + 1) * cfg.C].reshape(cfg.C, *kv)]).contiguous() for b in range(cfg.B)]
+        cv.set_prefix(new_pk, new_pv)
+        seeds2 = tuple(s + 100 for s in cfg.canvas_seeds)
+        cv.reset(seeds=seeds2)
+        cfg2 = fx.derive(cfg, canvas_seeds=seeds2, S=tuple(s + cfg.C for s in cfg.S))
+        rep2, steps2 = run_lockstep(cfg2, cv, m, om.append_block(m, pre, Ko, Vo), osched, sched, None)
+        assert not rep2.errors, "\n".join(rep2.errors[:20])
+        assert 1 <= steps2 <= cfg.max_steps
+    finally:
+        cv.close()
+
+
 def test_decode_block_matches_stepping():
     """dg_decode_block (device loop) ends in the same state as single steps."""
     from token_canvas_denoising_b200.canvas import from_workload, schedule

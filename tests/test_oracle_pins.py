@@ -392,6 +392,65 @@ def test_one_fixed_position_all_canvases_v2_c4(adaptive):
         assert final["tok"][0, 1] == init[1]
 
 
+# ---------------------------------------------------------------- blocks in sequence
+def _blk_cfg(dtype="bf16"):
+    return fx.Config(name="blk", B=2, C=5, S=(3, 0), d=16, Hq=2, Hk=1, h=8, V=32, dtype=dtype,
+                     max_steps=4, weight_seed=2, canvas_seeds=(3, 4))
+
+
+def test_block_kv_is_the_steps_canvas_kv():
+    cfg = _blk_cfg()
+    wl = fx.make_workload(cfg)
+    m = oracle_model(wl)
+    tok = oracle_init(wl)["tok"]
+    K, V = om.block_kv(m, tok)
+    _, _, _, ex = om.forward(m, oracle_prefix(wl), tok, None)
+    assert np.array_equal(K.reshape(ex["Kc"].shape), ex["Kc"])
+    assert np.array_equal(V.reshape(ex["Vc"].shape), ex["Vc"])
+
+
+def test_next_block_attends_to_prompt_then_committed_block():
+    """With Wq = 0 every score is 0, so block 2's attention output is the plain
+    mean of the request's prompt V rows, its committed block's V rows and its
+    own canvas V rows (a wrong tensor, request or order in the append fails)."""
+    cfg = _blk_cfg()
+    wl = fx.make_workload(cfg)
+    m = oracle_model(wl)
+    m["wq"] = np.zeros_like(m["wq"])
+    st1 = oracle_init(wl)
+    K1, V1 = om.block_kv(m, st1["tok"])
+    pre2 = om.append_block(m, oracle_prefix(wl), K1, V1)
+    tok2 = om.init_state(np.array([7, 8], dtype=np.uint64), cfg.C, cfg.V)["tok"]
+    _, _, _, ex = om.forward(m, pre2, tok2, None)
+    O = ex["O"].reshape(cfg.B, cfg.C, cfg.Hq, cfg.h)
+    _, V2 = om.block_kv(m, tok2)
+    for b in range(cfg.B):
+        rows = [om.widen(wl.prefix_v[b], cfg.dtype).reshape(-1, cfg.Hk, cfg.h), V1[b], V2[b]]
+        mean = np.concatenate(rows).mean(axis=0)[0]
+        want = on.round_to_bf16(np.broadcast_to(mean, (cfg.C, cfg.h)))
+        for q in range(cfg.Hq):
+            assert np.array_equal(O[b, :, q], want)
+        assert pre2[b][0].shape[0] == cfg.S[b] + cfg.C
+
+
+def test_two_blocks_in_sequence_keep_the_invariants():
+    cfg = fx.Config(name="two", B=1, C=4, S=(3,), d=8, Hq=2, Hk=1, h=4, V=8, dtype="f32",
+                    max_steps=3, weight_seed=11, canvas_seeds=(9,))
+    wl = fx.make_workload(cfg)
+    m = oracle_model(wl)
+    sched = oracle_sched(cfg, False)
+    st1 = oracle_init(wl)
+    fin1, recs1 = om.decode(m, oracle_prefix(wl), st1, sched)
+    _check_trajectory(cfg, st1, fin1, recs1, False)
+    K1, V1 = om.block_kv(m, fin1["tok"])
+    pre2 = om.append_block(m, oracle_prefix(wl), K1, V1)
+    cfg2 = fx.derive(cfg, canvas_seeds=(10,))
+    st2 = om.init_state(np.array([10], dtype=np.uint64), cfg.C, cfg.V)
+    fin2, recs2 = om.decode(m, pre2, st2, sched)
+    _check_trajectory(cfg2, st2, fin2, recs2, False)
+    assert pre2[0][0].shape[0] == cfg.S[0] + cfg.C
+
+
 # ---------------------------------------------------------------- MoE
 def _moe_cfg():
     return fx.Config(name="moe_t", B=1, C=5, S=(3,), d=12, Hq=2, Hk=1, h=4, V=16, dtype="f32",

@@ -53,6 +53,8 @@ SIGNATURES = {
     "dg_canvas_sync": (C.c_int, [C.c_void_p]),
     "dg_canvas_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
     "dg_canvas_reset_fixed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_canvas_block_kv": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_canvas_set_prefix": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_canvas_set_timing_events": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]),
     "dg_canvas_destroy": (None, [C.c_void_p]),
     "dg_status_string": (C.c_char_p, [C.c_int]),

@@ -138,6 +138,29 @@ class DenoiseCanvas:
                                              toks.ctypes.data_as(C.c_void_p))
         L.check(st, "dg_canvas_reset_fixed")
 
+    def block_kv(self):
+        """K and V of the current canvas tokens (the committed block), device
+        tensors [B*C, Hk*h] in the storage dtype, canvas-major."""
+        sdt = torch.float32 if self.dtype == "f32" else torch.bfloat16
+        kd = self._model.n_kv_heads * self._model.head_dim
+        dev = torch.device("cuda", torch.cuda.current_device())
+        k = torch.empty(self.M, kd, dtype=sdt, device=dev)
+        v = torch.empty(self.M, kd, dtype=sdt, device=dev)
+        st = self._lib.dg_canvas_block_kv(self._ctx, _ptr(k), _ptr(v))
+        L.check(st, "dg_canvas_block_kv")
+        return k, v
+
+    def set_prefix(self, prefix_k, prefix_v):
+        """Attend to new prompt caches from the next step on: lists of B device
+        tensors [S_b, Hk, h] (kept alive by this object)."""
+        plen = (C.c_int32 * self.B)(*[int(t.shape[0]) if t is not None else 0 for t in prefix_k])
+        pk = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_k])
+        pv = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_v])
+        st = self._lib.dg_canvas_set_prefix(self._ctx, C.cast(plen, C.c_void_p), C.cast(pk, C.c_void_p),
+                                            C.cast(pv, C.c_void_p))
+        L.check(st, "dg_canvas_set_prefix")
+        self._keep[1], self._keep[2] = prefix_k, prefix_v
+
     def set_timing_events(self, starts, stops):
         """Record torch.cuda.Event pairs around the LM-head kernel of graph steps
         (pair i on step i mod n). Pass empty lists to turn off."""

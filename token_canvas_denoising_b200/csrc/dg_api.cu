@@ -333,6 +333,7 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   if (model->dtype == DG_BF16) {
     c->lm.P = dg::lmhead_tc_partitions(c->M, model->vocab, c->ex.sm_count);
     c->attn_splits = dg::attn_tc_splits(batch, canvas_len, model->n_q_heads, c->S.data(), c->ex.sm_count);
+    c->attn_splits_cap = c->attn_splits;
     // tile / split choice only (buffers are bound after the workspace exists)
     const int qd = model->n_q_heads * model->head_dim, kd = model->n_kv_heads * model->head_dim;
     const void* wqkv[3] = {model->wq, model->wk, model->wv};
@@ -459,6 +460,65 @@ dg_status dg_canvas_reset_fixed(dg_ctx* ctx, const uint64_t* seeds, const uint8_
   DG_CUDA_RET(cudaMemcpyAsync(ctx->cs.frozen, frozen.data(), ctx->M, cudaMemcpyHostToDevice, ctx->ex.stream));
   DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
   return read_device_error(ctx);
+}
+
+dg_status dg_canvas_block_kv(dg_ctx* c, void* k_out, void* v_out) {
+  DG_ARG(c != nullptr, "ctx is NULL");
+  DG_ARG(k_out && v_out, "k_out / v_out is NULL");
+  const int M = c->M, d = c->m.d_model, V = c->m.vocab;
+  const int qd = c->m.n_q_heads * c->m.head_dim, kd = c->m.n_kv_heads * c->m.head_dim;
+  dg::Exec& ex = c->ex;
+  ex.launches = 0;
+  dg::launch_embed(ex, c->m.dtype, c->m.embed, c->cs.tok, c->X, M, d, V);
+  if (c->m.dtype == DG_BF16) {
+    dg::launch_gemm_tc(ex, c->g_qkv, nullptr);
+  } else {
+    dg::launch_linear_simple(ex, c->m.dtype, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
+    dg::launch_linear_simple(ex, c->m.dtype, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
+  }
+  (void)qd;
+  dg_status st = check_launch("block K/V");
+  if (st != DG_OK) return st;
+  DG_CUDA_RET(cudaMemcpyAsync(k_out, c->Kc, (size_t)M * kd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+  DG_CUDA_RET(cudaMemcpyAsync(v_out, c->Vc, (size_t)M * kd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+  return DG_OK;
+}
+
+dg_status dg_canvas_set_prefix(dg_ctx* c, const int32_t* prefix_len, const void* const* prefix_k,
+                               const void* const* prefix_v) {
+  DG_ARG(c != nullptr, "ctx is NULL");
+  DG_ARG(prefix_len != nullptr, "prefix_len is NULL");
+  for (int b = 0; b < c->B; ++b) {
+    DG_ARG(prefix_len[b] >= 0 && prefix_len[b] <= (1 << 24), "prefix_len out of range");
+    if (prefix_len[b] > 0) {
+      DG_ARG(prefix_k && prefix_v && prefix_k[b] && prefix_v[b], "prefix K/V pointer is NULL");
+      DG_ARG(aligned16(prefix_k[b]) && aligned16(prefix_v[b]), "prefix K/V must be 16-byte aligned");
+    }
+  }
+  DG_CUDA_RET(cudaStreamSynchronize(c->ex.stream));  // queued steps read the old prefix
+  drop_graphs(c);
+  c->max_S = 0;
+  for (int b = 0; b < c->B; ++b) {
+    c->S[b] = prefix_len[b];
+    c->pk[b] = prefix_len[b] ? prefix_k[b] : nullptr;
+    c->pv[b] = prefix_len[b] ? prefix_v[b] : nullptr;
+    c->max_S = std::max(c->max_S, (int)prefix_len[b]);
+  }
+  if (c->m.dtype == DG_BF16) {
+    // the split partial buffers were sized at init: never exceed that split count
+    c->attn_splits =
+        std::min(c->attn_splits_cap, dg::attn_tc_splits(c->B, c->C, c->m.n_q_heads, c->S.data(), c->ex.sm_count));
+    dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
+    if (!dg::attn_tc_prepare(&c->attn, sh, c->Q, c->Kc, c->Vc, c->S.data(), c->pk.data(), c->pv.data(), c->O,
+                             c->attn.part_o, c->attn.part_ml, c->attn_splits))
+      return DG_ERR_CUDA;
+  }
+  std::vector<dg::PrefixDesc> pd(c->B);
+  for (int b = 0; b < c->B; ++b) pd[b] = {c->pk[b], c->pv[b], c->S[b], 0};
+  DG_CUDA_RET(cudaMemcpyAsync(c->d_prefix, pd.data(), c->B * sizeof(dg::PrefixDesc), cudaMemcpyHostToDevice,
+                              c->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(c->ex.stream));
+  return DG_OK;
 }
 
 dg_status dg_decode_block(dg_ctx* ctx, const dg_schedule* sched, int32_t* tokens_out, int32_t* steps_out) {

@@ -204,6 +204,7 @@ struct dg_ctx {
   dg::GemmTc g_qkv, g_wo;
   dg::AttnTc attn;
   int attn_splits = 1;
+  int attn_splits_cap = 1;  // split partial buffers in the workspace are sized for this many
   dg::MoeTc moe;
   void* moe_ws = nullptr;
 

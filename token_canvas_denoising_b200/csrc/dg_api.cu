@@ -88,9 +88,7 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   }
   if (c->m.dtype == DG_BF16) {
     c->g_qkv.part = w.take<float>(dg::gemm_tc_partial_floats(c->g_qkv));
-    c->g_qkv.counters = w.take<unsigned>(dg::gemm_tc_counters(c->g_qkv));
     c->g_wo.part = w.take<float>(dg::gemm_tc_partial_floats(c->g_wo));
-    c->g_wo.counters = w.take<unsigned>(dg::gemm_tc_counters(c->g_wo));
   }
   if (c->m.dtype == DG_BF16 && c->attn_splits > 1) {
     const size_t rows = M * (size_t)c->m.n_q_heads;
@@ -379,15 +377,7 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
         !dg::gemm_tc_prepare(&c->g_wo, c->O, c->M, qd, 1, wo, oo, no, c->ex.sm_count))
       return fail(DG_ERR_CUDA);
     c->g_qkv.part = gq.part;
-    c->g_qkv.counters = gq.counters;
     c->g_wo.part = gw.part;
-    c->g_wo.counters = gw.counters;
-    if (c->g_qkv.counters &&
-        cudaMemsetAsync(c->g_qkv.counters, 0, dg::gemm_tc_counters(c->g_qkv) * sizeof(unsigned), c->ex.stream) != cudaSuccess)
-      return fail(DG_ERR_CUDA);
-    if (c->g_wo.counters &&
-        cudaMemsetAsync(c->g_wo.counters, 0, dg::gemm_tc_counters(c->g_wo) * sizeof(unsigned), c->ex.stream) != cudaSuccess)
-      return fail(DG_ERR_CUDA);
     dg::AttnShape sh{batch, canvas_len, model->n_q_heads, model->n_kv_heads, model->head_dim};
     if (!dg::attn_tc_prepare(&c->attn, sh, c->Q, c->Kc, c->Vc, c->S.data(), c->pk.data(), c->pv.data(), c->O,
                              c->attn.part_o, c->attn.part_ml, c->attn_splits))

@@ -414,7 +414,6 @@ bool gemm_tc_prepare(GemmTc* g, const void* A, int M, int K, int nseg, const voi
 size_t gemm_tc_partial_floats(const GemmTc& g) {
   return g.splits > 1 ? (size_t)g.splits * g.M * g.ncols : 0;
 }
-size_t gemm_tc_counters(const GemmTc&) { return 0; }
 
 void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual) {
   gemmtc::Params p;

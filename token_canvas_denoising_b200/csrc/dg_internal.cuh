@@ -94,17 +94,15 @@ struct alignas(64) GemmTc {
   void* out[3] = {nullptr, nullptr, nullptr};
   int N[3] = {0, 0, 0};
   float* part = nullptr;         // split-K partials [splits][M][ncols]
-  unsigned* counters = nullptr;  // per output tile, zero between launches
 };
 // Chooses the tile width and the K splits (for sm_count SMs) and encodes the
-// tensor maps; the caller then provides `part` and zeroed `counters` of the
-// sizes below when splits > 1.
+// tensor maps; the caller then provides `part` of the size below when
+// splits > 1.
 bool gemm_tc_prepare(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W, void* const* out,
                      const int* N, int sm_count);
 bool gemm_tc_prepare_with(GemmTc* g, const void* A, int M, int K, int nseg, const void* const* W,
                           void* const* out, const int* N, int bn, int splits);
 size_t gemm_tc_partial_floats(const GemmTc& g);
-size_t gemm_tc_counters(const GemmTc& g);
 void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual);
 
 // tcgen05 attention (bf16, head_dim 128): tensor maps per group of up to 8

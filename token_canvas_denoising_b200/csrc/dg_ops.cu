@@ -143,18 +143,11 @@ dg_status dg_linear(int32_t dtype, const void* a, const void* w, const void* res
     const int ns[1] = {N};
     if (!dg::gemm_tc_prepare(&g, a, M, K, 1, ws, os, ns, ex.sm_count)) return DG_ERR_CUDA;
     void* tmp = nullptr;
-    const size_t pf = dg::gemm_tc_partial_floats(g), nc = dg::gemm_tc_counters(g);
+    const size_t pf = dg::gemm_tc_partial_floats(g);
     if (g.splits > 1) {
-      dg_status st = cuda_status(cudaMallocAsync(&tmp, pf * sizeof(float) + nc * sizeof(unsigned), ex.stream),
-                                 "cudaMallocAsync");
+      dg_status st = cuda_status(cudaMallocAsync(&tmp, pf * sizeof(float), ex.stream), "cudaMallocAsync");
       if (st != DG_OK) return st;
       g.part = static_cast<float*>(tmp);
-      g.counters = reinterpret_cast<unsigned*>(g.part + pf);
-      st = cuda_status(cudaMemsetAsync(g.counters, 0, nc * sizeof(unsigned), ex.stream), "cudaMemsetAsync");
-      if (st != DG_OK) {
-        cudaFreeAsync(tmp, ex.stream);
-        return st;
-      }
     }
     dg::launch_gemm_tc(ex, g, residual);
     if (tmp) cudaFreeAsync(tmp, ex.stream);

@@ -76,6 +76,14 @@ dg_status dg_attention(int32_t dtype, const void *q, const void *kc, const void 
 dg_status dg_linear(int32_t dtype, const void *a, const void *w, const void *residual, void *out,
                     int32_t M, int32_t N, int32_t K, void *stream);
 
+/* Failure-detection self-test (no counterpart in the pages): one CTA waits on
+ * a barrier that nothing completes, through the same bounded wait every kernel
+ * of the step uses. The wait gives up after its limit (2 s), records a timeout
+ * in a device error word and the kernel returns; the call then returns
+ * DG_ERR_TIMEOUT, leaving the CUDA context usable. Synchronous. Anything else
+ * (DG_OK included) means the bounded-wait path is broken. */
+dg_status dg_selftest_wait_timeout(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

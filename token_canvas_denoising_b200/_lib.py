@@ -54,6 +54,7 @@ SIGNATURES = {
     "dg_canvas_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
     "dg_canvas_reset_fixed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_canvas_block_kv": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_selftest_wait_timeout": (C.c_int, [C.c_void_p]),
     "dg_canvas_set_prefix": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_canvas_set_timing_events": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]),
     "dg_canvas_destroy": (None, [C.c_void_p]),

@@ -83,6 +83,42 @@ def test_init_rejects_bad_models(lib, over, status):
     assert not ctx.value
 
 
+_BF16 = dict(dtype=1, head_dim=128, vocab=1024, d_model=128)
+_MOE = dict(n_experts=32, top_k=4, moe_inter=128, n_shared=1, w_router=4096, w_gate=4096, w_up=4096,
+            w_down=4096)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(_MOE), 2),                                   # MoE needs the bf16 storage dtype
+    (dict(_BF16, **dict(_MOE, n_experts=48)), 2),      # a multiple of 32 experts
+    (dict(_BF16, **dict(_MOE, top_k=9, n_experts=64)), 2),
+    (dict(_BF16, **dict(_MOE, top_k=33)), 1),          # top_k > n_experts
+    (dict(_BF16, **dict(_MOE, moe_inter=100)), 2),
+    (dict(_BF16, **dict(_MOE, n_shared=3)), 2),
+    (dict(_BF16, **dict(_MOE, w_up=None)), 1),
+])
+def test_init_rejects_bad_moe_models(lib, over, status):
+    m = _model(**over)
+    ctx = C.c_void_p()
+    plen = (C.c_int32 * 1)(0)
+    seeds = (C.c_uint64 * 1)(0)
+    st = lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None,
+                            None, C.cast(seeds, C.c_void_p), None)
+    assert st == status, lib.dg_last_error()
+    assert not ctx.value
+
+
+def test_init_rejects_moe_beyond_one_routing_block(lib):
+    m = _model(**dict(_BF16, **_MOE))
+    ctx = C.c_void_p()
+    plen = (C.c_int32 * 2)(0, 0)
+    seeds = (C.c_uint64 * 2)(0, 1)
+    st = lib.dg_canvas_init(C.byref(ctx), C.byref(m), 2, 200, C.cast(plen, C.c_void_p), None, None,
+                            None, C.cast(seeds, C.c_void_p), None)
+    assert st == 2 and b"256" in lib.dg_last_error()
+    assert not ctx.value
+
+
 @pytest.mark.parametrize("batch,canvas", [(0, 16), (1, 0), (1, 257)])
 def test_init_rejects_bad_sizes(lib, batch, canvas):
     m = _model()
@@ -100,6 +136,11 @@ def test_null_context_calls_fail_cleanly(lib):
     assert lib.dg_denoise_step(None, C.byref(s), None) == 1
     assert lib.dg_decode_block(None, C.byref(s), None, None) == 1
     assert lib.dg_canvas_sync(None) == 1
+    mask = (C.c_uint8 * 4)()
+    toks = (C.c_int32 * 4)()
+    assert lib.dg_canvas_reset_fixed(None, None, C.cast(mask, C.c_void_p), C.cast(toks, C.c_void_p)) == 1
+    assert lib.dg_canvas_block_kv(None, None, None) == 1
+    assert lib.dg_canvas_set_prefix(None, None, None, None) == 1
     lib.dg_canvas_destroy(None)
 
 

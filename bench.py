@@ -191,9 +191,11 @@ def bench_reference(args, rank, world):
     full step (embed, Q/K/V, attention over the whole prefix, Wo + residual, LM
     head over the whole vocabulary, entropy/argmax, freeze, re-noise) on the
     first r canvas positions only, r chosen so that warm-up + timed steps fit
-    in about REF_BUDGET_S seconds (from a two-point cost model measured first).
-    The workload's steps/s is reported as (sample steps/s) * r / C. Weights and
-    prefix K/V are widened to fp64 once, before the timed region."""
+    in about REF_BUDGET_S seconds. A cost model t(r) = a + b r is calibrated
+    first from one step on 1 row and one step on the whole canvas; the
+    workload's step time is the measured sample step time plus (C - r) rows at
+    the per-row cost b. Weights and prefix K/V are widened to fp64 once, before
+    the timed region."""
     if rank != 0:
         return 0
     from oracle import model as om
@@ -216,18 +218,26 @@ def bench_reference(args, rank, world):
                 st = om.init_state(wl.seeds, rows, cfg.V)
         return time.perf_counter() - t0
 
-    # cost model t(r) = a + b r from r = 1 and r = 16
+    # per-step cost t(r) = a + b r (a: work independent of the sampled rows,
+    # such as streaming the weights; b: per row), from one step on 1 row and
+    # one step on the whole canvas, so the model is exact at both ends
+    tc0 = time.perf_counter()
     t1 = run(1, 2) / 2
-    t16 = run(min(16, cfg.C), 2) / 2
-    b = max(0.0, (t16 - t1) / max(1, min(16, cfg.C) - 1))
+    tC = run(cfg.C, 1) if cfg.C > 1 else t1
+    b = max(0.0, (tC - t1) / max(1, cfg.C - 1))
     a = max(1e-4, t1 - b)
-    per_step = REF_BUDGET_S / max(1, args.steps + args.warmup)
+    budget = max(10.0, REF_BUDGET_S - (time.perf_counter() - tc0))
+    per_step = budget / max(1, args.steps + args.warmup)
     rows = int(max(1, min(cfg.C, (per_step - a) / b if b > 0 else cfg.C)))
     run(rows, args.warmup)
     dt = run(rows, args.steps)
-    v = args.steps / dt * rows / cfg.C
+    # a full step costs the measured sample step plus the remaining rows at the
+    # measured per-row cost
+    t_full = dt / args.steps + b * (cfg.C - rows)
+    v = 1.0 / t_full
     sample = (f"{args.steps} oracle denoise steps (fp64 numpy) on the first {rows} of {cfg.C} canvas positions "
-              f"of the {cfg.name} workload (full prefix, full vocabulary), steps/s scaled by {rows}/{cfg.C}")
+              f"of the {cfg.name} workload (full prefix, full vocabulary); full-step time = measured sample "
+              f"step time + {cfg.C - rows} rows x the measured per-row cost ({b * 1e3:.3f} ms)")
     line = {"impl": "reference", "metric": "denoise steps/s", "value": v, "unit": "steps/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",

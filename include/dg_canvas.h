@@ -117,6 +117,9 @@ typedef struct dg_step_out {
   void *hidden;         /* [B*C][d_model] residual stream fed to the LM head   */
   void *hidden_attn;    /* [B*C][d_model] residual stream after attention and Wo,
                            before the MoE block (equals `hidden` without MoE)  */
+  void *q;              /* [B*C][n_q_heads*head_dim] queries (dtype)           */
+  void *k_canvas;       /* [B*C][n_kv_heads*head_dim] canvas keys (dtype)      */
+  void *v_canvas;       /* [B*C][n_kv_heads*head_dim] canvas values (dtype)    */
 } dg_step_out;
 
 /* Host-side copy of the decode state (all host arrays). */

@@ -158,16 +158,24 @@ def gelu_exact(x):
     return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
 
 
-def moe_route(model, Hs):
+def moe_route(model, Hs, choice=None):
     """Router logits, softmax, top-k by probability (lower expert index first on
-    ties), gates renormalised over the chosen experts. Returns (logits, idx, gates)."""
+    ties), gates renormalised over the chosen experts. Returns (logits, idx, gates).
+
+    choice: optional [rows, k] expert indices used instead of the top-k (to
+    evaluate another valid choice where the k-th and (k+1)-th probabilities of
+    a row are tied within the comparison tolerance); the gates are still the
+    softmax probabilities of the chosen experts renormalised over them."""
     dt = model["dtype"]
     r = Hs @ widen(model["w_router"], dt).T
     p = softmax_rows(r)
     k = model["top_k"]
     E = p.shape[1]
-    # stable sort on -p keeps the lower index first among equal probabilities
-    order = np.argsort(-p, axis=1, kind="stable")[:, :k]
+    if choice is None:
+        # stable sort on -p keeps the lower index first among equal probabilities
+        order = np.argsort(-p, axis=1, kind="stable")[:, :k]
+    else:
+        order = np.asarray(choice, dtype=np.int64).reshape(p.shape[0], k)
     gp = np.take_along_axis(p, order, axis=1)
     gates = gp / np.sum(gp, axis=1, keepdims=True)
     assert E == model["n_experts"]
@@ -183,10 +191,11 @@ def expert_ffn(model, e, x):
     return a @ widen(model["w_down"][e], dt).T
 
 
-def moe_block(model, Hs):
-    """Hs + sum_e gate_e FFN_e(Hs) + sum_shared FFN_shared(Hs), rounded to storage."""
+def moe_block(model, Hs, choice=None):
+    """Hs + sum_e gate_e FFN_e(Hs) + sum_shared FFN_shared(Hs), rounded to storage.
+    choice: optional expert indices per row (see moe_route)."""
     dt = model["dtype"]
-    r, idx, gates = moe_route(model, Hs)
+    r, idx, gates = moe_route(model, Hs, choice)
     E = model["n_experts"]
     out = np.zeros_like(Hs)
     for e in range(E):

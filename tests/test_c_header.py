@@ -15,7 +15,8 @@ STRUCTS = {
     "dg_model_desc": ["d_model", "vocab", "dtype", "embed", "lm_head", "n_experts", "n_shared", "w_router",
                       "w_down"],
     "dg_schedule": ["max_steps", "stop_entropy", "adaptive_stop", "kind"],
-    "dg_step_out": ["ent", "argmax", "freeze_mask", "attn_out", "hidden", "hidden_attn"],
+    "dg_step_out": ["ent", "argmax", "freeze_mask", "attn_out", "hidden", "hidden_attn", "q", "k_canvas",
+                    "v_canvas"],
     "dg_state": ["tokens", "frozen", "step", "seed", "done"],
 }
 

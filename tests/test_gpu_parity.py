@@ -36,6 +36,7 @@ def _run(cfg, adaptive=True, n_steps=None, free_running=True, check_tensors=True
                                   check_tensors=check_tensors)
     finally:
         cv.close()
+    print(f"{cfg.name}: {steps} steps; {rep.summary()}")
     assert not rep.errors, "\n".join(rep.errors[:20])
     return rep, steps
 
@@ -58,9 +59,10 @@ def test_bf16_small_multi_tile():
     _run(cfg, n_steps=4)
 
 
-def test_bf16_canvas256_first_steps():
+def test_bf16_canvas256_first_steps_lockstep():
     """The canvas256 workload (B1 C256 S1024 d2048 16/8 heads, V32768): the
-    first steps in lock-step against the oracle."""
+    first steps in lock-step (the GPU restarts every step from the oracle's
+    state) against the oracle."""
     _run(fx.CONFIGS["canvas256"], n_steps=3, free_running=False)
 
 

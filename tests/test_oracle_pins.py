@@ -497,6 +497,77 @@ def test_moe_identical_experts_reduce_to_single_ffn():
     assert np.allclose(out, on.round_to_f32(Hs + 2.0 * y), rtol=1e-6, atol=1e-6)
 
 
+def _gate_pairing_model(router_logits):
+    """Three routed experts, top-2, no shared expert, d = 4, I = 1, f32 storage.
+    The token is the unit vector e_0, so the router logits are column 0 of
+    W_router. Every expert has the same gate and up rows (the same scalar
+    activation a), and expert e writes only coordinate e + 1, scaled by
+    c_e = e + 1: FFN_e(e_0) = a c_e e_{e+1}."""
+    E, d = 3, 4
+    m = {"dtype": "f32", "d": d, "n_experts": E, "top_k": 2, "moe_inter": 1, "n_shared": 0}
+    wr = np.zeros((E, d), np.float32)
+    wr[:, 0] = router_logits
+    m["w_router"] = wr
+    m["w_gate"] = np.zeros((E, 1, d), np.float32)
+    m["w_gate"][:, 0, 0] = 1.5
+    m["w_up"] = np.zeros((E, 1, d), np.float32)
+    m["w_up"][:, 0, 0] = 1.0
+    m["w_down"] = np.zeros((E, d, 1), np.float32)
+    for e in range(E):
+        m["w_down"][e, e + 1, 0] = e + 1.0
+    return m
+
+
+@pytest.mark.parametrize("logits,chosen", [((2.0, 1.0, 0.0), (0, 1)), ((0.0, 1.0, 2.0), (2, 1)),
+                                           ((1.0, -3.0, 2.0), (2, 0))])
+def test_moe_gate_pairing_with_distinct_experts(logits, chosen):
+    """Each expert's output is weighted by its own gate. With router logits
+    r_i > r_j for the two chosen experts, the renormalised gates are
+    e^(r_i) / (e^(r_i) + e^(r_j)) and e^(r_j) / (...), so the contributions on
+    the experts' own coordinates, divided by c_e, stand in the ratio
+    e^(r_i - r_j) (for logits 2 and 1: exactly e), sum to the shared activation
+    a, and the unchosen expert's coordinate stays 0. Pairing each expert with
+    another slot's gate inverts the ratio."""
+    m = _gate_pairing_model(logits)
+    x = np.zeros((1, 4))
+    x[0, 0] = 1.0
+    out, (r, idx, gates) = om.moe_block(m, x)
+    assert sorted(idx[0].tolist()) == sorted(chosen)
+    y = out[0] - x[0]
+    contrib = {e: y[e + 1] / (e + 1.0) for e in range(3)}
+    i, j = chosen
+    assert contrib[i] / contrib[j] == pytest.approx(math.exp(logits[i] - logits[j]), rel=1e-6)
+    unchosen = ({0, 1, 2} - set(chosen)).pop()
+    assert y[unchosen + 1] == 0.0
+    # the two contributions add up to the common activation a = GELU(1.5) * 1
+    assert contrib[i] + contrib[j] == pytest.approx(1.5 * 0.5 * (1.0 + math.erf(1.5 / math.sqrt(2.0))), rel=1e-6)
+
+
+def test_moe_explicit_choice_uses_the_chosen_experts_gates():
+    """Routing a row to another valid pair of experts (as the parity harness
+    does where the k-th and (k+1)-th router logits are tied within its
+    tolerance) renormalises the softmax over that pair."""
+    m = _gate_pairing_model((2.0, 1.0, 0.0))
+    x = np.zeros((1, 4))
+    x[0, 0] = 1.0
+    out, (_, idx, gates) = om.moe_block(m, x, choice=[[0, 2]])
+    assert idx[0].tolist() == [0, 2]
+    assert gates[0] == pytest.approx([math.exp(2) / (math.exp(2) + 1), 1 / (math.exp(2) + 1)], rel=1e-12)
+    y = out[0] - x[0]
+    assert y[2] == 0.0 and (y[1] / 1.0) / (y[3] / 3.0) == pytest.approx(math.exp(2.0), rel=1e-6)
+
+
+def test_planted_swapped_moe_gates_are_caught(monkeypatch):
+    real = om.moe_route
+
+    def swapped(model, Hs, choice=None):
+        r, idx, gates = real(model, Hs, choice)
+        return r, idx, gates[:, ::-1].copy()
+    monkeypatch.setattr(om, "moe_route", swapped)
+    with pytest.raises(AssertionError):
+        test_moe_gate_pairing_with_distinct_experts((2.0, 1.0, 0.0), (0, 1))
+
+
 def test_gelu_matches_torch_exact():
     x = np.linspace(-6, 6, 101)
     ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="none").numpy()

@@ -33,7 +33,8 @@ class dg_schedule(C.Structure):
 
 class dg_step_out(C.Structure):
     _fields_ = [("ent", C.c_void_p), ("argmax", C.c_void_p), ("freeze_mask", C.c_void_p),
-                ("attn_out", C.c_void_p), ("hidden", C.c_void_p), ("hidden_attn", C.c_void_p)]
+                ("attn_out", C.c_void_p), ("hidden", C.c_void_p), ("hidden_attn", C.c_void_p),
+                ("q", C.c_void_p), ("k_canvas", C.c_void_p), ("v_canvas", C.c_void_p)]
 
 
 class dg_state(C.Structure):

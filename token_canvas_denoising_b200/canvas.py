@@ -76,6 +76,8 @@ class DenoiseCanvas:
         if debug:
             dev = torch.device("cuda", torch.cuda.current_device())
             sdt = torch.float32 if self.dtype == "f32" else torch.bfloat16
+            qd = self._model.n_q_heads * self._model.head_dim
+            kd = self._model.n_kv_heads * self._model.head_dim
             out = {
                 "ent": torch.empty(self.M, dtype=torch.float32, device=dev),
                 "argmax": torch.empty(self.M, dtype=torch.int32, device=dev),
@@ -83,9 +85,12 @@ class DenoiseCanvas:
                 "attn_out": torch.empty(self.M, self._model.n_q_heads * self._model.head_dim, dtype=sdt, device=dev),
                 "hidden": torch.empty(self.M, self._model.d_model, dtype=sdt, device=dev),
                 "hidden_attn": torch.empty(self.M, self._model.d_model, dtype=sdt, device=dev),
+                "q": torch.empty(self.M, qd, dtype=sdt, device=dev),
+                "k_canvas": torch.empty(self.M, kd, dtype=sdt, device=dev),
+                "v_canvas": torch.empty(self.M, kd, dtype=sdt, device=dev),
             }
             dbg = L.dg_step_out(*[_ptr(out[k]) for k in ("ent", "argmax", "freeze_mask", "attn_out", "hidden",
-                                                          "hidden_attn")])
+                                                          "hidden_attn", "q", "k_canvas", "v_canvas")])
         st = self._lib.dg_denoise_step(self._ctx, C.byref(sched), C.byref(dbg) if dbg is not None else None)
         L.check(st, "dg_denoise_step")
         return out

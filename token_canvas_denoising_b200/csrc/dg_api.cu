@@ -193,6 +193,11 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
     if (dbg->hidden) DG_CUDA_RET(cudaMemcpyAsync(dbg->hidden, hs, (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, ex.stream));
     if (dbg->hidden_attn)
       DG_CUDA_RET(cudaMemcpyAsync(dbg->hidden_attn, c->Hs, (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->q) DG_CUDA_RET(cudaMemcpyAsync(dbg->q, c->Q, (size_t)M * qd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->k_canvas)
+      DG_CUDA_RET(cudaMemcpyAsync(dbg->k_canvas, c->Kc, (size_t)M * kd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->v_canvas)
+      DG_CUDA_RET(cudaMemcpyAsync(dbg->v_canvas, c->Vc, (size_t)M * kd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
   }
   return DG_OK;
 }

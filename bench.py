@@ -1,7 +1,7 @@
 """Throughput of the canvas denoise step on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload canvas256]
+                    [--workload longctx]
 
 A bench step is one denoise step: every row of the hot path (embed, Q/K/V
 projection, bidirectional attention over prefix + canvas, Wo + residual, LM
@@ -11,11 +11,16 @@ whole batch of canvases, run as one CUDA-graph launch through the C ABI. Every
 so each timed step does real freezing work. Inputs are synthetic and seeded;
 the weights and prefix K/V are resident in HBM before the timed region.
 
+The default workload is the largest that fits one GPU: longctx, four canvases
+of 256 positions, each over its own 32,768-token prompt K/V, vocabulary
+262,144 (1.82 TFLOP and 2.1 GB of weights and K/V per step).
+
 Multi-GPU: the canvases are independent requests, so N ranks run N replicas
 with no data-path collective (weak scaling); the reported time is the max over
 ranks and the value counts the steps of every rank.
 """
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -29,6 +34,10 @@ sys.path.insert(0, ROOT)
 
 BLOCK_STEPS = 48
 REF_BUDGET_S = 150.0  # target wall time of the whole reference-arm run
+# per workload: (timed steps, warm-up steps, e2e decode blocks) when not given
+DEFAULTS = {"tiny": (4800, 96, 20), "canvas256": (4800, 96, 20), "vocab262k": (480, 48, 4),
+            "longctx": (240, 24, 2), "moe": (480, 48, 4)}
+SUSTAINED_AFTER_S = 1.0  # a kernel timed over a region at least this long takes the sustained peak
 
 
 # ---------------------------------------------------------------- ranks
@@ -59,13 +68,18 @@ def rank_canvas_seeds(seeds, rank):
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4800)
-    ap.add_argument("--warmup", type=int, default=96)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", default="canvas256")
-    ap.add_argument("--e2e-blocks", type=int, default=20)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    return ap.parse_args()
+    ap.add_argument("--workload", default="longctx")
+    ap.add_argument("--e2e-blocks", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    a = ap.parse_args()
+    st, wu, eb = DEFAULTS.get(a.workload, (480, 48, 4))
+    a.steps = st if a.steps is None else a.steps
+    a.warmup = wu if a.warmup is None else a.warmup
+    a.e2e_blocks = eb if a.e2e_blocks is None else a.e2e_blocks
+    return a
 
 
 def load_peaks():
@@ -133,8 +147,21 @@ def workload_cfg(name):
     return fx.CONFIGS[name]
 
 
+def workload_label(cfg):
+    moe = (f", MoE {cfg.n_experts}+{cfg.n_shared} experts top-{cfg.top_k} I{cfg.moe_inter}"
+           if cfg.n_experts else "")
+    return (f"{cfg.name}: B{cfg.B} C{cfg.C} S{cfg.S[0]} d{cfg.d} Hq{cfg.Hq}/Hk{cfg.Hk} h{cfg.h} V{cfg.V} "
+            f"{cfg.dtype}{moe}, {cfg.max_steps}-step blocks, adaptive stop off")
+
+
 def flops_bytes(cfg):
-    """Algorithmic flops and HBM bytes of one step and of the LM-head kernel."""
+    """Algorithmic flops and HBM bytes of one step and of the two gated kernels.
+
+    LM head: 2 M d V flops; bytes = the weights once + Hs once + one 32-byte
+    partial record per (row, vocab partition) written (about 148 per 256 rows,
+    counted as 148 per row here as an upper bound on that small term).
+    Attention: 4 C (S + C) h Hq flops per request; bytes = the prompt K/V once,
+    Q, the canvas K/V and O."""
     M, d, V = cfg.B * cfg.C, cfg.d, cfg.V
     qd, kd = cfg.Hq * cfg.h, cfg.Hk * cfg.h
     es = 2 if cfg.dtype == "bf16" else 4
@@ -143,10 +170,17 @@ def flops_bytes(cfg):
     f_attn = sum(4 * cfg.C * (s + cfg.C) * cfg.h * cfg.Hq for s in cfg.S)
     f_wo = 2 * M * qd * d
     f_lm = 2 * M * d * V
-    b_lm = V * d * es + M * d * es + M * 32  # W once, Hs once, one 32-byte record per row... per CTA
-    b_step = ((qd + 2 * kd) * d + d * qd + V * d) * es + 2 * S * kd * es + M * d * es * 6
-    return {"flops_step": f_qkv + f_attn + f_wo + f_lm, "bytes_step": b_step, "flops_lm": f_lm,
-            "bytes_lm_weights": V * d * es}
+    f_moe = 0
+    b_moe = 0
+    if cfg.n_experts:
+        I = cfg.moe_inter
+        f_moe = 2 * M * d * cfg.n_experts + M * (cfg.top_k + cfg.n_shared) * 6 * d * I
+        b_moe = (cfg.n_experts + cfg.n_shared) * 3 * d * I * es + cfg.n_experts * d * es
+    b_lm = V * d * es + M * d * es + M * 148 * 32
+    b_attn = 2 * S * kd * es + M * (2 * qd + 2 * kd) * es
+    b_step = ((qd + 2 * kd) * d + d * qd + V * d) * es + 2 * S * kd * es + M * d * es * 6 + b_moe
+    return {"flops_step": f_qkv + f_attn + f_wo + f_lm + f_moe, "bytes_step": b_step,
+            "flops_lm": f_lm, "bytes_lm": b_lm, "flops_attn": f_attn, "bytes_attn": b_attn}
 
 
 def cpu_cores_used():
@@ -160,56 +194,30 @@ def cpu_cores_used():
     return os.cpu_count()
 
 
-def run_oracle_sample(cfg, seconds, wl=None):
-    """Time the fp64 oracle's denoise steps on this host for about `seconds`.
-    Returns (steps/s, steps run, sample description)."""
-    from oracle import model as om
-    from token_canvas_denoising_b200 import inputs as fx
-    wl = wl or fx.make_workload(cfg)
+def oracle_model_of(cfg, wl):
+    """The oracle's model dictionary for a workload (MoE weights included)."""
     m = {"dtype": cfg.dtype, "d": cfg.d, "Hq": cfg.Hq, "Hk": cfg.Hk, "h": cfg.h, "V": cfg.V}
     m.update({k: wl.weights[k] for k in ("embed", "wq", "wk", "wv", "wo", "lm_head")})
-    prefix = list(zip(wl.prefix_k, wl.prefix_v))
-    sched = {"max_steps": cfg.max_steps, "stop_entropy": cfg.stop_entropy, "adaptive_stop": False}
-    invT = None if cfg.inv_temp == "one" else wl.inv_temp
-    st = om.init_state(wl.seeds, cfg.C, cfg.V)
-    n = 0
-    t0 = time.perf_counter()
-    while True:
-        st, _ = om.denoise_step(m, prefix, st, sched, invT)
-        n += 1
-        if time.perf_counter() - t0 >= seconds or bool(st["done"].all()):
-            break
-    dt = time.perf_counter() - t0
-    return n / dt, n, f"{n} full oracle denoise steps of the {cfg.name} workload (fp64, numpy)"
+    if cfg.n_experts:
+        m.update(n_experts=cfg.n_experts, top_k=cfg.top_k, moe_inter=cfg.moe_inter, n_shared=cfg.n_shared)
+        m.update({k: wl.weights[k] for k in ("w_router", "w_gate", "w_up", "w_down")})
+    return m
 
 
-# ---------------------------------------------------------------- reference arm
-def bench_reference(args, rank, world):
-    """The fp64 oracle on this host's cores, on the same workload and unit.
-
-    Each reference step is a bounded sample of one denoise step: the oracle's
-    full step (embed, Q/K/V, attention over the whole prefix, Wo + residual, LM
-    head over the whole vocabulary, entropy/argmax, freeze, re-noise) on the
-    first r canvas positions only, r chosen so that warm-up + timed steps fit
-    in about REF_BUDGET_S seconds. A cost model t(r) = a + b r is calibrated
-    first from one step on 1 row and one step on the whole canvas; the
-    workload's step time is the measured sample step time plus (C - r) rows at
-    the per-row cost b. Weights and prefix K/V are widened to fp64 once, before
-    the timed region."""
-    if rank != 0:
-        return 0
+def oracle_step_timer(cfg, wl):
+    """run(rows, n): wall time of n oracle denoise steps (adaptive stop off)
+    on the first `rows` positions of every canvas of the workload, restarting
+    the block when it is done. Weights and prefix K/V are widened to fp64
+    first (outside the timed calls)."""
     from oracle import model as om
-    from token_canvas_denoising_b200 import inputs as fx
-    cfg = workload_cfg(args.workload)
-    wl = fx.make_workload(cfg)
-    m = {"dtype": cfg.dtype, "d": cfg.d, "Hq": cfg.Hq, "Hk": cfg.Hk, "h": cfg.h, "V": cfg.V}
-    m.update({k: wl.weights[k] for k in ("embed", "wq", "wk", "wv", "wo", "lm_head")})
-    m = om.prewiden(m)
+    m = om.prewiden(oracle_model_of(cfg, wl))
     prefix = [(om.widen(k, cfg.dtype), om.widen(v, cfg.dtype)) for k, v in zip(wl.prefix_k, wl.prefix_v)]
     sched = {"max_steps": cfg.max_steps, "stop_entropy": cfg.stop_entropy, "adaptive_stop": False}
 
     def run(rows, n):
-        invT = None if cfg.inv_temp == "one" else wl.inv_temp[:rows]
+        invT = None
+        if cfg.inv_temp != "one":
+            invT = wl.inv_temp.reshape(cfg.B, cfg.C)[:, :rows].reshape(-1)
         st = om.init_state(wl.seeds, rows, cfg.V)
         t0 = time.perf_counter()
         for _ in range(n):
@@ -217,34 +225,87 @@ def bench_reference(args, rank, world):
             if st["done"].all():
                 st = om.init_state(wl.seeds, rows, cfg.V)
         return time.perf_counter() - t0
+    return run
 
-    # per-step cost t(r) = a + b r (a: work independent of the sampled rows,
-    # such as streaming the weights; b: per row), from one step on 1 row and
-    # one step on the whole canvas, so the model is exact at both ends
+
+def oracle_rate(cfg, wl, budget_s, n_steps=None, n_warm=0):
+    """The fp64 oracle's denoise steps/s on this host, within about budget_s.
+
+    A per-step cost model t(r) = a + b r (a: work independent of the sampled
+    rows, such as streaming the widened weights; b: per canvas row) is
+    calibrated from steps on 1 row and on r2 = min(C, 16) rows. When a full
+    step fits the budget, full steps are timed; otherwise steps on the first r
+    rows of every canvas (r as large as the budget allows) are timed and the
+    full-step time is the measured sample step plus (C - r) rows at the
+    per-row cost b (the sampled rows attend to S + r keys instead of S + C;
+    the prompt dominates the keys of the large workloads).
+    Returns (steps/s, description of the sample)."""
+    run = oracle_step_timer(cfg, wl)
     tc0 = time.perf_counter()
     t1 = run(1, 2) / 2
-    tC = run(cfg.C, 1) if cfg.C > 1 else t1
-    b = max(0.0, (tC - t1) / max(1, cfg.C - 1))
+    r2 = min(cfg.C, 16)
+    t2 = run(r2, 1) if r2 > 1 else t1
+    b = max(0.0, (t2 - t1) / max(1, r2 - 1))
     a = max(1e-4, t1 - b)
-    budget = max(10.0, REF_BUDGET_S - (time.perf_counter() - tc0))
-    per_step = budget / max(1, args.steps + args.warmup)
+    left = max(5.0, budget_s - (time.perf_counter() - tc0))
+    n = n_steps or max(1, int(left / max(1e-3, a + b * cfg.C)))
+    per_step = left / max(1, n + n_warm)
     rows = int(max(1, min(cfg.C, (per_step - a) / b if b > 0 else cfg.C)))
-    run(rows, args.warmup)
-    dt = run(rows, args.steps)
-    # a full step costs the measured sample step plus the remaining rows at the
-    # measured per-row cost
-    t_full = dt / args.steps + b * (cfg.C - rows)
-    v = 1.0 / t_full
-    sample = (f"{args.steps} oracle denoise steps (fp64 numpy) on the first {rows} of {cfg.C} canvas positions "
-              f"of the {cfg.name} workload (full prefix, full vocabulary); full-step time = measured sample "
-              f"step time + {cfg.C - rows} rows x the measured per-row cost ({b * 1e3:.3f} ms)")
+    if n_warm:
+        run(rows, n_warm)
+    dt = run(rows, n)
+    t_full = dt / n + b * (cfg.C - rows)
+    if rows == cfg.C:
+        sample = (f"{n} full oracle denoise steps (fp64 numpy) of the {cfg.name} workload "
+                  f"({cfg.B} x {cfg.C} positions)")
+    else:
+        sample = (f"{n} oracle denoise steps (fp64 numpy) on the first {rows} of {cfg.C} positions of each of the "
+                  f"{cfg.B} canvas(es) of the {cfg.name} workload (full prompt, full vocabulary); full-step time = "
+                  f"measured sample step + {cfg.C - rows} rows x the per-row cost ({b * 1e3:.2f} ms/row, "
+                  f"calibrated on 1- and {r2}-row steps)")
+    return 1.0 / t_full, sample
+
+
+def source_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_of(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu
+    summary, or None when there is none or the kernel's source changed since."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{kernel}_{workload}.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        if t.get("source_sha256_16") != source_sha(t["source"]):
+            return None
+        return t.get("bytes_per_launch")
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- reference arm
+def bench_reference(args, rank, world):
+    """The fp64 oracle on this host's cores, on the same workload and unit.
+
+    Each reference step is a bounded sample of one denoise step (see
+    oracle_rate): the oracle's full step (embed, Q/K/V, attention over the
+    whole prompt, Wo + residual (+ MoE), LM head over the whole vocabulary,
+    entropy/argmax, freeze, re-noise) on the first r canvas positions, r
+    chosen so that warm-up + timed steps fit in about REF_BUDGET_S seconds."""
+    if rank != 0:
+        return 0
+    from token_canvas_denoising_b200 import inputs as fx
+    cfg = workload_cfg(args.workload)
+    wl = fx.make_workload(cfg)
+    v, sample = oracle_rate(cfg, wl, REF_BUDGET_S, n_steps=args.steps, n_warm=args.warmup)
     line = {"impl": "reference", "metric": "denoise steps/s", "value": v, "unit": "steps/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "canvas_tokens_per_s": v * cfg.B * cfg.C,
-            "config": {"workload": f"{cfg.name}: B{cfg.B} C{cfg.C} S{cfg.S[0]} d{cfg.d} Hq{cfg.Hq}/Hk{cfg.Hk} "
-                                   f"h{cfg.h} V{cfg.V} {cfg.dtype}, {cfg.max_steps}-step blocks, adaptive stop off"},
+            "config": {"workload": workload_label(cfg)},
             "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cpu_cores_used(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -253,6 +314,21 @@ def bench_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------- b200 arm
+def kernel_roofline(name, kernel, flops, bytes_, avg_ms, peaks, peak_kind, traffic):
+    peak = peaks["bf16_tflops_sustained"] if peak_kind == "sustained" else peaks["bf16_tflops"]
+    tflops = flops / (avg_ms / 1e3) / 1e12
+    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    return {"bound": "tensor", "kernel": kernel, "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+            "frac": tflops / peak, "traffic": traffic,
+            "peak_source": f"{peaks['source']} {peak_kind} bf16 ("
+                           + ("kernel timed inside a step loop of a second or more"
+                              if peak_kind == "sustained" else "kernel timed inside a step loop shorter than 1 s")
+                           + ")",
+            "avg_ms": avg_ms, "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": bytes_,
+            "hbm_bound_ms": bytes_ / (peaks["hbm_gbs"] * 1e9) * 1e3, "roofline_ms": t_roof,
+            "frac_of_roofline_time": t_roof / avg_ms}
+
+
 def bench_b200(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -303,46 +379,61 @@ def bench_b200(args, rank, world, local_rank):
     t_stop.record(stream)
     torch.cuda.synchronize()
     elapsed_ms = t_start.elapsed_time(t_stop)
-    ck = clocks.stop()
     cv.sync()
     n_resets = (args.steps - 1) // BLOCK_STEPS
     if world > 1:
         elapsed_ms = max_over_ranks(elapsed_ms, world, "cuda")
         dist.barrier()
 
-    # ---- timed region 2: the same steps with CUDA events recorded around the
-    # LM-head kernel on its stream (a ring of NEV event pairs, one graph
-    # variant each); gives the dominant kernel's average launch duration
+    # ---- timed region 2: the same steps with CUDA events recorded on the
+    # step's stream around the LM-head kernel and around the attention kernel
+    # (rings of NEV event pairs, one graph variant each): the gated kernels'
+    # average launch durations
     NEV = 4
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(NEV)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(NEV)]
-    for e in ev_s + ev_e:  # torch creates the CUDA event on its first record
-        e.record(stream)
-    cv.set_timing_events(ev_s, ev_e)
+    ev = {k: ([torch.cuda.Event(enable_timing=True) for _ in range(NEV)],
+              [torch.cuda.Event(enable_timing=True) for _ in range(NEV)]) for k in ("lmhead", "attention")}
+    for s_, e_ in ev.values():
+        for e in s_ + e_:  # torch creates the CUDA event on its first record
+            e.record(stream)
+    for k, (s_, e_) in ev.items():
+        cv.set_timing_events(s_, e_, kernel=k)
     cv.reset()
     run_steps(NEV, 0)  # capture every variant before timing
     cv.sync()
     cv.reset()
-    lm_steps = min(args.steps, 960)
-    lm_ms = []
-    for i in range(lm_steps):
+    k_steps = min(args.steps, 960)
+    dur = {k: [] for k in ev}
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for i in range(k_steps):
         if i % BLOCK_STEPS == 0 and i > 0:
             cv.reset()
         cv.step(sched)
         j = i - (NEV - 1)
-        if j >= 0:  # the pair used NEV-1 steps ago: wait for it (NEV-1 steps stay queued)
-            ev_e[j % NEV].synchronize()
-            lm_ms.append(ev_s[j % NEV].elapsed_time(ev_e[j % NEV]))
+        if j >= 0:  # the pairs used NEV-1 steps ago: wait for them (NEV-1 steps stay queued)
+            for k, (s_, e_) in ev.items():
+                e_[j % NEV].synchronize()
+                dur[k].append(s_[j % NEV].elapsed_time(e_[j % NEV]))
+    r1.record(stream)
     torch.cuda.synchronize()
-    for j in range(max(0, lm_steps - (NEV - 1)), lm_steps):
-        lm_ms.append(ev_s[j % NEV].elapsed_time(ev_e[j % NEV]))
-    cv.set_timing_events([], [])
+    for j in range(max(0, k_steps - (NEV - 1)), k_steps):
+        for k, (s_, e_) in ev.items():
+            dur[k].append(s_[j % NEV].elapsed_time(e_[j % NEV]))
+    region2_s = r0.elapsed_time(r1) / 1e3
+    ck = clocks.stop()
+    for k in ev:
+        cv.set_timing_events([], [], kernel=k)
     steps_per_s = job_rate(args.steps, world, elapsed_ms)
-    lm_avg_ms = float(np.mean(lm_ms))
-    lm_tflops = fb["flops_lm"] / (lm_avg_ms / 1e3) / 1e12
+    peak_kind = "sustained" if region2_s >= SUSTAINED_AFTER_S else "burst"
+    lm = kernel_roofline("lmhead", "lmhead_tc_kernel (LM head + entropy/argmax)", fb["flops_lm"], fb["bytes_lm"],
+                         float(np.mean(dur["lmhead"])), peaks, peak_kind, traffic_of("lmhead_tc_kernel", cfg.name))
+    at = kernel_roofline("attention", "attn_tc_kernel (+ attn_merge_kernel when split)", fb["flops_attn"],
+                         fb["bytes_attn"], float(np.mean(dur["attention"])), peaks, peak_kind,
+                         traffic_of("attn_tc_kernel", cfg.name))
 
     # ---- end to end through the C ABI with host buffers: per block, the initial
-    # state goes host->device (pinned) and the tokens come back device->host
+    # state goes host->device (pinned), dg_decode_block runs the block's steps
+    # (its loop on the device) and the tokens come back device->host
     e2e = None
     if rank == 0 or world > 1:
         cv.reset()  # a fresh block: step 0, nothing frozen
@@ -351,7 +442,7 @@ def bench_b200(args, rank, world, local_rank):
         pin_np = {k: v.numpy() for k, v in pin.items()}
         tok_out = torch.empty(cfg.B * cfg.C, dtype=torch.int32).pin_memory()
         cv.set_state(pin_np)
-        cv.decode(sched, tok_out)  # warm
+        cv.decode(sched, tok_out)  # warm (builds the decode graph)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         total_steps = 0
@@ -376,27 +467,17 @@ def bench_b200(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1:
-        v, n, sample = run_oracle_sample(cfg, args.cpu_seconds, wl)
+        v, sample = oracle_rate(cfg, wl, args.cpu_seconds)
         cpu = {"value": v, "unit": "steps/s", "cores": cpu_cores_used(), "kind": "oracle", "sample": sample}
 
     if rank == 0:
-        traffic = None
-        tpath = os.path.join(ROOT, "profiles", f"lmhead_traffic_{cfg.name}.json")
-        if os.path.exists(tpath):
-            try:
-                with open(tpath) as f:
-                    traffic = json.load(f).get("bytes_per_launch")
-            except Exception:
-                traffic = None
-        peak = peaks["bf16_tflops_sustained"]
         line = {
             "metric": "denoise steps/s", "value": steps_per_s, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
             "data": "synthetic",
             "canvas_tokens_per_s": steps_per_s * cfg.B * cfg.C,
-            "config": {"workload": f"{cfg.name}: B{cfg.B} C{cfg.C} S{cfg.S[0]} d{cfg.d} Hq{cfg.Hq}/Hk{cfg.Hk} "
-                                   f"h{cfg.h} V{cfg.V} {cfg.dtype}, {cfg.max_steps}-step blocks, adaptive stop off",
+            "config": {"workload": workload_label(cfg),
                        "batch_canvases": cfg.B, "canvas_len": cfg.C, "prefix_len": cfg.S[0],
                        "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: each step streams {fb['bytes_step'] / 1e6:.0f} MB of weights "
@@ -404,18 +485,15 @@ def bench_b200(args, rank, world, local_rank):
             "clocks": ck,
             "e2e": e2e,
             "gpu_launches": int(args.steps * launches_per_step + n_resets),
-            "roofline": {"bound": "tensor", "kernel": "lmhead_tc_kernel (LM head + entropy/argmax)",
-                         "achieved": lm_tflops, "peak": peak, "unit": "TFLOP/s", "frac": lm_tflops / peak,
-                         "traffic": traffic,
-                         "peak_source": f"{peaks['source']} sustained bf16 (kernel timed inside a long step loop)",
-                         "avg_ms": lm_avg_ms,
-                         "algorithmic_flops_per_launch": fb["flops_lm"],
-                         "hbm_bound_ms": fb["bytes_lm_weights"] / (peaks["hbm_gbs"] * 1e9) * 1e3},
+            "roofline": lm,
+            "rooflines": {"lmhead": lm, "attention": at},
             "step_roofline": {"flops": fb["flops_step"], "bytes": fb["bytes_step"],
                               "ms": max(fb["flops_step"] / (peaks["bf16_tflops"] * 1e12),
                                         fb["bytes_step"] / (peaks["hbm_gbs"] * 1e9)) * 1e3},
+            "kernel_timing_region_s": region2_s,
             "cpu_baseline": cpu,
         }
+        line["step_roofline"]["frac"] = line["step_roofline"]["ms"] / line["ms_per_step"]
         print(json.dumps(line), flush=True)
     cv.close()
     return 0

@@ -202,8 +202,12 @@ dg_status dg_canvas_set_prefix(dg_ctx *ctx, const int32_t *prefix_len, const voi
 /* Denoise until every canvas is done (at most sched->max_steps steps each).
  *   tokens_out  [B*C] int32, device or host memory (copied with UVA), or NULL.
  *   steps_out   host [B] steps taken per canvas, or NULL.
- * Synchronous. The loop runs on the device (a CUDA graph with a device-side
- * stop flag); the host reads one flag per step batch. */
+ * Synchronous. The loop runs on the device: one CUDA graph launch, whose
+ * conditional while node repeats the step until the step's selection kernel
+ * finds every canvas done (no step runs after that); the host waits once.
+ * The first call with a given schedule builds that graph, so it must not
+ * happen inside a stream capture. A canvas still open after max_steps steps
+ * (impossible under DG_SCHED_CEIL) ends the loop with DG_ERR_DEVICE_CHECK. */
 dg_status dg_decode_block(dg_ctx *ctx, const dg_schedule *sched, int32_t *tokens_out,
                           int32_t *steps_out);
 
@@ -216,8 +220,16 @@ dg_status dg_canvas_set_state(dg_ctx *ctx, const dg_state *host_in);
 /* Timing support: with n > 0 pairs of CUDA events (cudaEvent_t, created by the
  * caller with timing enabled), step number i (counted from this call) of
  * dg_denoise_step without debug outputs records starts[i % n] just before and
- * stops[i % n] just after the LM-head kernel. n = 0 turns it off.
- * Synchronous (drops the captured step graphs). */
+ * stops[i % n] just after the kernel named by `kernel`: DG_KERNEL_LMHEAD (the
+ * LM head with its entropy/argmax epilogue) or DG_KERNEL_ATTENTION (the
+ * attention kernel, with its split-KV merge when it has one). n = 0 turns it
+ * off for that kernel; the two kernels' settings are independent.
+ * Synchronous (drops the captured step graphs). Not used by dg_decode_block. */
+#define DG_KERNEL_LMHEAD 0
+#define DG_KERNEL_ATTENTION 1
+dg_status dg_canvas_set_kernel_timing(dg_ctx *ctx, int32_t kernel, int32_t n, void *const *starts,
+                                      void *const *stops);
+/* dg_canvas_set_kernel_timing(ctx, DG_KERNEL_LMHEAD, n, starts, stops). */
 dg_status dg_canvas_set_timing_events(dg_ctx *ctx, int32_t n, void *const *starts, void *const *stops);
 
 /* Wait for the context's stream and report device-side errors (synchronous). */

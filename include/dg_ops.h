@@ -8,9 +8,10 @@
  * All pointers are device memory unless marked host; all matrices row-major;
  * dtype is DG_F32 or DG_BF16 (the storage type of every non-f32 buffer).
  * Each call queues work on `stream` (cudaStream_t, NULL = default), allocates
- * and frees its own temporary buffers (stream-ordered), and returns DG_OK or
- * an error status (see dg_canvas.h); dg_last_error() has the detail. The
- * calls do not synchronize.
+ * and frees its own temporary buffers (stream-ordered; except
+ * dg_lmhead_entropy_noalloc), and returns DG_OK or an error status (see
+ * dg_canvas.h); dg_last_error() has the detail. The calls do not synchronize;
+ * dg_ops_check reports what went wrong on the device.
  */
 #ifndef DG_OPS_H
 #define DG_OPS_H
@@ -35,22 +36,25 @@ dg_status dg_lmhead_entropy(int32_t dtype, const void *hs, const void *lm_head, 
                             int32_t M, int32_t d, int32_t V, float *ent, int32_t *argmax, void *stream);
 
 /* Allocation-free variant of dg_lmhead_entropy. The pages have no counterpart
- * to this call: it exists for users of this library who may not allocate
- * device memory at the point where they run the LM head -- work that is being
- * recorded into a CUDA graph, or an application whose device memory is
- * reserved up front by its own allocator.
- * Same arguments and results as dg_lmhead_entropy. Its temporary per-row
- * partial results go to a fixed device array inside the library (2 MiB, held
- * on every GPU that loads the library until the process exits) instead of a
+ * to this call: it exists for callers of this library that cannot allocate
+ * device memory where they run the LM head -- an application whose device
+ * memory is reserved up front by its own allocator (a driver allocation in
+ * the middle of a step would fail or fragment what is left), or a host that
+ * gives a plug-in only the buffers it passes and forbids it to allocate.
+ * Same arguments and results as dg_lmhead_entropy (the same kernels with the
+ * same vocab partitions, so the same bits). Its temporary per-row partial
+ * results go to a fixed device array inside the library (2 MiB, held on
+ * every GPU that loads the library until the process exits) instead of a
  * fresh buffer; the call makes no cudaMalloc, cudaFree or other allocation.
  * Limit: M times the number of vocab partitions (at most the GPU's SM count,
  * fewer for M > 256) must not exceed dg_lmhead_entropy_noalloc_max_records()
- * (65,536); larger problems return DG_ERR_UNSUPPORTED.
- * The first call on each device looks up the array's device address; make
- * that first call before any stream capture. All calls on a device share the
- * array: two calls whose work can overlap on the GPU (e.g. on different
- * streams without ordering between them) race. Nothing in the array needs to
- * start at zero: each call writes every entry it reads. */
+ * (65,536); larger problems return DG_ERR_UNSUPPORTED before any work.
+ * The first call on each device (and CUDA context) looks up the array's
+ * device address; make that first call before any stream capture. All calls
+ * on a device share the array: two calls whose work can overlap on the GPU
+ * (e.g. on different streams without ordering between them) race. Nothing in
+ * the array needs to start at zero: each call writes every entry it reads.
+ * Device-side failures are reported by dg_ops_check. */
 dg_status dg_lmhead_entropy_noalloc(int32_t dtype, const void *hs, const void *lm_head,
                                     const float *inv_temp, int32_t M, int32_t d, int32_t V,
                                     float *ent, int32_t *argmax, void *stream);
@@ -75,6 +79,15 @@ dg_status dg_attention(int32_t dtype, const void *q, const void *kc, const void 
  * re-projected every step). bf16 needs K % 64 == 0 and N % 64 == 0. */
 dg_status dg_linear(int32_t dtype, const void *a, const void *w, const void *residual, void *out,
                     int32_t M, int32_t N, int32_t K, void *stream);
+
+/* Device-side status of the calls above: waits for `stream` and reports the
+ * first device-side failure any of their kernels recorded since the last
+ * dg_ops_check -- DG_ERR_TIMEOUT when a bounded wait inside a kernel gave up
+ * (its outputs are then not valid), DG_ERR_DEVICE_CHECK for a failed data
+ * check (a NaN entropy) -- and clears it. DG_OK when none failed.
+ * Synchronous. The calls above only validate their arguments and queue work;
+ * their return status cannot include what happens on the device. */
+dg_status dg_ops_check(void* stream);
 
 /* Failure-detection self-test (no counterpart in the pages): one CTA waits on
  * a barrier that nothing completes, through the same bounded wait every kernel

@@ -29,7 +29,7 @@ def _program():
              "  fn volatile f[] = {(fn)dg_canvas_init, (fn)dg_denoise_step, (fn)dg_decode_block,",
              "                     (fn)dg_canvas_reset_fixed, (fn)dg_canvas_block_kv, (fn)dg_canvas_set_prefix,",
              "                     (fn)dg_lmhead_entropy, (fn)dg_lmhead_entropy_noalloc, (fn)dg_attention,",
-             "                     (fn)dg_linear, (fn)dg_selftest_wait_timeout};",
+             "                     (fn)dg_linear, (fn)dg_ops_check, (fn)dg_selftest_wait_timeout};",
              "  (void)f;"]
     for s, fields in STRUCTS.items():
         lines.append(f'  printf("{s} size %zu\\n", sizeof({s}));')

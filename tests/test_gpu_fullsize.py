@@ -25,27 +25,28 @@ from tests.parity import abi_state_to_oracle, run_lockstep
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-_WIDE = {}
+_CACHE = {}
 
 
-def _oracle(wl):
-    """The oracle model with its dense weights widened to fp64 once per workload."""
-    name = wl.cfg.name
-    if name not in _WIDE:
-        _WIDE.clear()
-        _WIDE[name] = om.prewiden(oracle_model(wl))
-    return _WIDE[name]
+def _workload(name):
+    """The seeded workload and the oracle model over it (dense weights widened
+    to fp64 once), kept for the tests of the same workload."""
+    if name not in _CACHE:
+        _CACHE.clear()
+        wl = fx.make_workload(fx.CONFIGS[name])
+        _CACHE[name] = (wl, om.prewiden(oracle_model(wl)))
+    return _CACHE[name]
 
 
 def _decode(name, adaptive):
     from token_canvas_denoising_b200.canvas import from_workload, schedule
     cfg = fx.CONFIGS[name]
-    wl = fx.make_workload(cfg)
+    wl, m = _workload(name)
     cv, keep = from_workload(wl)
     try:
         invT = None if cfg.inv_temp == "one" else wl.inv_temp.astype(np.float64)
         last = cfg.max_steps - 1
-        rep, steps = run_lockstep(cfg, cv, _oracle(wl), oracle_prefix(wl), oracle_sched(cfg, adaptive=adaptive),
+        rep, steps = run_lockstep(cfg, cv, m, oracle_prefix(wl), oracle_sched(cfg, adaptive=adaptive),
                                   schedule(cfg.max_steps, cfg.stop_entropy, adaptive), invT,
                                   free_running=True, check_tensors=True, tensor_steps={0, 1, 2, last})
         final = cv.get_state()
@@ -82,8 +83,8 @@ def test_moe_full_decode(adaptive):
 def test_longctx_first_steps_and_last_step():
     from token_canvas_denoising_b200.canvas import from_workload, schedule
     cfg = fx.CONFIGS["longctx"]
-    wl = fx.make_workload(cfg)
-    m, pre = _oracle(wl), oracle_prefix(wl)
+    wl, m = _workload("longctx")
+    pre = oracle_prefix(wl)
     sched, osched = schedule(cfg.max_steps, cfg.stop_entropy, False), oracle_sched(cfg, adaptive=False)
     cv, keep = from_workload(wl)
     try:

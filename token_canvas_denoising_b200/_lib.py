@@ -13,6 +13,7 @@ DG_OK, DG_ERR_INVALID_ARG, DG_ERR_UNSUPPORTED, DG_ERR_OOM, DG_ERR_CUDA, DG_ERR_T
     DG_ERR_DEVICE_CHECK = range(7)
 DG_F32, DG_BF16 = 0, 1
 DG_SCHED_CEIL = 0
+DG_KERNEL_LMHEAD, DG_KERNEL_ATTENTION = 0, 1
 
 
 class dg_model_desc(C.Structure):
@@ -58,6 +59,7 @@ SIGNATURES = {
     "dg_selftest_wait_timeout": (C.c_int, [C.c_void_p]),
     "dg_canvas_set_prefix": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_canvas_set_timing_events": (C.c_int, [C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]),
+    "dg_canvas_set_kernel_timing": (C.c_int, [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p]),
     "dg_canvas_destroy": (None, [C.c_void_p]),
     "dg_status_string": (C.c_char_p, [C.c_int]),
     "dg_last_error": (C.c_char_p, []),
@@ -74,6 +76,7 @@ SIGNATURES = {
                                C.c_void_p, C.c_void_p]),
     "dg_linear": (C.c_int, [C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
                             C.c_int32, C.c_int32, C.c_void_p]),
+    "dg_ops_check": (C.c_int, [C.c_void_p]),
 }
 
 _lib = None

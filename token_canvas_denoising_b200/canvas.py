@@ -166,14 +166,16 @@ class DenoiseCanvas:
         L.check(st, "dg_canvas_set_prefix")
         self._keep[1], self._keep[2] = prefix_k, prefix_v
 
-    def set_timing_events(self, starts, stops):
-        """Record torch.cuda.Event pairs around the LM-head kernel of graph steps
-        (pair i on step i mod n). Pass empty lists to turn off."""
+    def set_timing_events(self, starts, stops, kernel="lmhead"):
+        """Record torch.cuda.Event pairs around one kernel of graph steps
+        (pair i on step i mod n): kernel "lmhead" or "attention". Pass empty
+        lists to turn off."""
+        k = {"lmhead": L.DG_KERNEL_LMHEAD, "attention": L.DG_KERNEL_ATTENTION}[kernel]
         n = len(starts)
         a = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in starts])
         b = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in stops])
-        st = self._lib.dg_canvas_set_timing_events(self._ctx, n, C.cast(a, C.c_void_p), C.cast(b, C.c_void_p))
-        L.check(st, "dg_canvas_set_timing_events")
+        st = self._lib.dg_canvas_set_kernel_timing(self._ctx, k, n, C.cast(a, C.c_void_p), C.cast(b, C.c_void_p))
+        L.check(st, "dg_canvas_set_kernel_timing")
 
     def sync(self):
         L.check(self._lib.dg_canvas_sync(self._ctx), "dg_canvas_sync")

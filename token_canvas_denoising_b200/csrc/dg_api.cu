@@ -70,6 +70,7 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   c->cs.done = w.take<uint8_t>(c->B);
   c->cs.all_done = w.take<int32_t>(1);
   c->cs.counters = w.take<uint32_t>(c->B + 1);
+  c->cs.loop_iter = w.take<int32_t>(1);
   c->err = w.take<int32_t>(1);
   c->d_prefix = w.take<dg::PrefixDesc>(c->B);
   c->X = w.take<char>(M * d * c->es);
@@ -162,10 +163,15 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
     dg::launch_linear_simple(ex, dt, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
   }
   dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
+  // inside a stream capture, only an "external" record becomes an event node
+  if (c->cur_ev_start[DG_KERNEL_ATTENTION])
+    DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start[DG_KERNEL_ATTENTION], ex.stream, cudaEventRecordExternal));
   if (dt == DG_BF16)
     dg::launch_attn_tc(ex, c->attn);
   else
     dg::launch_attention_simple(ex, dt, c->Q, c->d_prefix, c->Kc, c->Vc, c->O, sh);
+  if (c->cur_ev_stop[DG_KERNEL_ATTENTION])
+    DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_stop[DG_KERNEL_ATTENTION], ex.stream, cudaEventRecordExternal));
   if (dt == DG_BF16)
     dg::launch_gemm_tc(ex, c->g_wo, c->X);
   else
@@ -175,14 +181,16 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
     dg::launch_moe(ex, c->moe);
     hs = c->Hs2;
   }
-  // inside a stream capture, only an "external" record becomes an event node
-  if (c->cur_ev_start) DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start, ex.stream, cudaEventRecordExternal));
+  if (c->cur_ev_start[DG_KERNEL_LMHEAD])
+    DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start[DG_KERNEL_LMHEAD], ex.stream, cudaEventRecordExternal));
   if (dt == DG_BF16)
     dg::launch_lmhead_tc(ex, c->tm_lm_a, c->tm_lm_b, c->lm, c->inv_temp, M, d, V);
   else
     dg::launch_lmhead_simple(ex, dt, hs, c->m.lm_head, c->inv_temp, c->lm, M, d, V);
-  if (c->cur_ev_stop) DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_stop, ex.stream, cudaEventRecordExternal));
-  dg::launch_merge_select(ex, c->lm, c->ent, c->am, dbg ? dbg->freeze_mask : nullptr, &c->cs, &s, c->B, c->C, V);
+  if (c->cur_ev_stop[DG_KERNEL_LMHEAD])
+    DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_stop[DG_KERNEL_LMHEAD], ex.stream, cudaEventRecordExternal));
+  dg::launch_merge_select(ex, c->lm, c->ent, c->am, dbg ? dbg->freeze_mask : nullptr, &c->cs, &s, c->B, c->C, V,
+                          c->cur_loop);
   c->launches = ex.launches;
   dg_status st = check_launch("denoise step launch");
   if (st != DG_OK) return st;
@@ -211,15 +219,96 @@ void drop_graphs(dg_ctx* c) {
   for (auto g : c->graphs)
     if (g) cudaGraphExecDestroy(g);
   c->graphs.clear();
+  if (c->decode_graph) cudaGraphExecDestroy(c->decode_graph);
+  c->decode_graph = nullptr;
+}
+
+// dg_decode_block's graph: a memset node clears the loop's step counter, then
+// a conditional while node runs the step (the same launch sequence as a graph
+// step, captured into the node's body) until the selection kernel of the step
+// that leaves every canvas done sets the condition to 0. The loop never runs
+// more than max_steps steps: every canvas stops by then (the freeze count
+// takes all remaining positions at its last step), and the kernel also ends
+// the loop at the cap (recording kDevLoopCap if a canvas is still open).
+// The body is captured with programmatic launches first, and without them if
+// the conditional body does not take them.
+dg_status build_decode_graph(dg_ctx* c, const dg_schedule& s) {
+  if (c->decode_graph && same_sched(c->decode_sched, s)) return DG_OK;
+  if (c->decode_graph) cudaGraphExecDestroy(c->decode_graph);
+  c->decode_graph = nullptr;
+  if (!c->capture_stream) DG_CUDA_RET(cudaStreamCreateWithFlags(&c->capture_stream, cudaStreamNonBlocking));
+  std::string why;
+  for (int attempt = 0; attempt < 2 && !c->decode_graph; ++attempt) {
+    cudaGraph_t g = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    cudaError_t e = cudaGraphCreate(&g, 0);
+    cudaGraphConditionalHandle h = 0;
+    if (e == cudaSuccess) e = cudaGraphConditionalHandleCreate(&h, g, 1, cudaGraphCondAssignDefault);
+    cudaGraphNode_t reset = nullptr, loop = nullptr;
+    if (e == cudaSuccess) {
+      cudaMemsetParams mp = {};
+      mp.dst = c->cs.loop_iter;
+      mp.value = 0;
+      mp.elementSize = 4;
+      mp.width = 1;
+      mp.height = 1;
+      mp.pitch = 4;
+      e = cudaGraphAddMemsetNode(&reset, g, nullptr, 0, &mp);
+    }
+    cudaGraphNodeParams cp = {};
+    if (e == cudaSuccess) {
+      cp.type = cudaGraphNodeTypeConditional;
+      cp.conditional.handle = h;
+      cp.conditional.type = cudaGraphCondTypeWhile;
+      cp.conditional.size = 1;
+      e = cudaGraphAddNode(&loop, g, &reset, 1, &cp);
+    }
+    dg_status st = DG_OK;
+    if (e == cudaSuccess) {
+      cudaGraph_t body = cp.conditional.phGraph_out[0];
+      cudaStream_t user = c->ex.stream;
+      c->ex.stream = c->capture_stream;
+      c->loop.handle = h;
+      c->loop.cap = s.max_steps;
+      c->cur_loop = &c->loop;
+      dg::t_pdl_off = attempt == 1;
+      e = cudaStreamBeginCaptureToGraph(c->capture_stream, body, nullptr, nullptr, 0,
+                                        cudaStreamCaptureModeThreadLocal);
+      if (e == cudaSuccess) {
+        st = enqueue_step(c, s, nullptr);
+        cudaGraph_t out = nullptr;
+        const cudaError_t e2 = cudaStreamEndCapture(c->capture_stream, &out);
+        if (e2 != cudaSuccess) e = e2;
+      }
+      dg::t_pdl_off = false;
+      c->cur_loop = nullptr;
+      c->ex.stream = user;
+    }
+    if (e == cudaSuccess && st == DG_OK) e = cudaGraphInstantiate(&exec, g, 0);
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    if (st != DG_OK) return st;
+    if (e == cudaSuccess) {
+      c->decode_graph = exec;
+      c->decode_sched = s;
+    } else {
+      why += std::string(attempt ? "; without programmatic launch: " : "") + cudaGetErrorString(e);
+    }
+  }
+  if (!c->decode_graph) {
+    set_last_error("building the device-side decode loop failed: " + why);
+    return DG_ERR_CUDA;
+  }
+  return DG_OK;
 }
 
 // One step without debug outputs: a CUDA graph of the whole launch sequence,
 // captured on a private stream the first time (and again when the schedule
 // changes), then launched on the caller's stream. With timing events set,
-// graph variant i records event pair i around the LM-head kernel, and step n
-// uses variant n mod (number of pairs).
+// graph variant i records, for each timed kernel k, event pair i mod n_k
+// around that kernel, and step n uses variant n mod (largest n_k).
 dg_status launch_step_graph(dg_ctx* c, const dg_schedule& s) {
-  const size_t nvar = std::max<size_t>(1, c->ev_start.size());
+  const size_t nvar = std::max<size_t>(1, std::max(c->ev_start[0].size(), c->ev_start[1].size()));
   if (c->graphs.size() != nvar || !same_sched(c->graph_sched, s)) {
     drop_graphs(c);
     c->graphs.assign(nvar, nullptr);
@@ -230,8 +319,11 @@ dg_status launch_step_graph(dg_ctx* c, const dg_schedule& s) {
     if (!c->capture_stream) DG_CUDA_RET(cudaStreamCreateWithFlags(&c->capture_stream, cudaStreamNonBlocking));
     cudaStream_t user = c->ex.stream;
     c->ex.stream = c->capture_stream;
-    c->cur_ev_start = c->ev_start.empty() ? nullptr : c->ev_start[v];
-    c->cur_ev_stop = c->ev_stop.empty() ? nullptr : c->ev_stop[v];
+    for (int k = 0; k < 2; ++k) {
+      const size_t nk = c->ev_start[k].size();
+      c->cur_ev_start[k] = nk ? c->ev_start[k][v % nk] : nullptr;
+      c->cur_ev_stop[k] = nk ? c->ev_stop[k][v % nk] : nullptr;
+    }
     cudaGraph_t g = nullptr;
     cudaError_t e = cudaStreamBeginCapture(c->capture_stream, cudaStreamCaptureModeThreadLocal);
     dg_status st = DG_OK;
@@ -240,7 +332,7 @@ dg_status launch_step_graph(dg_ctx* c, const dg_schedule& s) {
       e = cudaStreamEndCapture(c->capture_stream, &g);
     }
     c->ex.stream = user;
-    c->cur_ev_start = c->cur_ev_stop = nullptr;
+    for (int k = 0; k < 2; ++k) c->cur_ev_start[k] = c->cur_ev_stop[k] = nullptr;
     if (st != DG_OK) {
       if (g) cudaGraphDestroy(g);
       return st;
@@ -520,22 +612,16 @@ dg_status dg_decode_block(dg_ctx* ctx, const dg_schedule* sched, int32_t* tokens
   DG_ARG(ctx != nullptr, "ctx is NULL");
   dg_status st = validate_sched(sched);
   if (st != DG_OK) return st;
-  // Every canvas stops within max_steps (the freeze count reaches all
-  // remaining positions at the last step), so max_steps launches suffice; the
-  // device flag lets the host stop early without a per-step round trip.
+  // One launch of the decode graph: the loop over steps and its end run on
+  // the device. The host only looks at the done flag first (a block that is
+  // already finished launches nothing).
   int32_t all = 0;
   DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->cs.all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->ex.stream));
   DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
-  int launched = 0;
-  while (!all && launched < sched->max_steps) {
-    const int batch = std::min(4, sched->max_steps - launched);
-    for (int i = 0; i < batch; ++i) {
-      st = launch_step_graph(ctx, *sched);
-      if (st != DG_OK) return st;
-    }
-    launched += batch;
-    DG_CUDA_RET(cudaMemcpyAsync(&all, ctx->cs.all_done, sizeof(all), cudaMemcpyDeviceToHost, ctx->ex.stream));
-    DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
+  if (!all) {
+    st = build_decode_graph(ctx, *sched);
+    if (st != DG_OK) return st;
+    DG_CUDA_RET(cudaGraphLaunch(ctx->decode_graph, ctx->ex.stream));
   }
   st = read_device_error(ctx);
   if (st != DG_OK) return st;
@@ -579,21 +665,27 @@ dg_status dg_canvas_set_state(dg_ctx* ctx, const dg_state* h) {
   return DG_OK;
 }
 
-dg_status dg_canvas_set_timing_events(dg_ctx* ctx, int32_t n, void* const* starts, void* const* stops) {
+dg_status dg_canvas_set_kernel_timing(dg_ctx* ctx, int32_t kernel, int32_t n, void* const* starts,
+                                      void* const* stops) {
   DG_ARG(ctx != nullptr, "ctx is NULL");
+  DG_ARG(kernel == DG_KERNEL_LMHEAD || kernel == DG_KERNEL_ATTENTION, "unknown kernel id");
   DG_ARG(n >= 0 && n <= 64, "n must be in [0, 64]");
   if (n > 0) DG_ARG(starts && stops, "event arrays are NULL");
   for (int i = 0; i < n; ++i) DG_ARG(starts[i] && stops[i], "NULL event");
   DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
   drop_graphs(ctx);
-  ctx->ev_start.clear();
-  ctx->ev_stop.clear();
+  ctx->ev_start[kernel].clear();
+  ctx->ev_stop[kernel].clear();
   for (int i = 0; i < n; ++i) {
-    ctx->ev_start.push_back(static_cast<cudaEvent_t>(starts[i]));
-    ctx->ev_stop.push_back(static_cast<cudaEvent_t>(stops[i]));
+    ctx->ev_start[kernel].push_back(static_cast<cudaEvent_t>(starts[i]));
+    ctx->ev_stop[kernel].push_back(static_cast<cudaEvent_t>(stops[i]));
   }
   ctx->step_launch_count = 0;
   return DG_OK;
+}
+
+dg_status dg_canvas_set_timing_events(dg_ctx* ctx, int32_t n, void* const* starts, void* const* stops) {
+  return dg_canvas_set_kernel_timing(ctx, DG_KERNEL_LMHEAD, n, starts, stops);
 }
 
 dg_status dg_canvas_sync(dg_ctx* ctx) {

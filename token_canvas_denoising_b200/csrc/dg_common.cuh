@@ -17,6 +17,7 @@ enum DeviceError : int {
   kDevWaitTimeout = 3,   // a bounded mbarrier wait gave up
   kDevBadShape = 4,      // a kernel was launched on shapes it does not support
   kDevBadAlign = 5,      // shared memory not aligned as a kernel's tile layout needs
+  kDevLoopCap = 6,       // a device-side decode loop reached its step cap with a canvas not done
 };
 
 __device__ __forceinline__ void set_error(int* err, int code) {

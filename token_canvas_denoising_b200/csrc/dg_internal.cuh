@@ -3,6 +3,7 @@
 #pragma once
 #include <cuda.h>
 
+#include <mutex>
 #include <string>
 #include <utility>
 #include <vector>
@@ -50,9 +51,67 @@ struct AttnShape {
 
 void set_last_error(const std::string& msg);
 
+// The calling thread's current CUDA context (dg_tmap.cu).
+bool current_context(void** ctx);
+
+// Device addresses of one file-scope __device__ variable, one per (device,
+// context). In host code the variable's name is only a host-side stand-in,
+// so its address on the current device is looked up with
+// cudaGetSymbolAddress the first time a context uses it, and kept. Keying on
+// the context makes an address looked up before a device reset (which ends
+// that context) unreachable afterwards. get() must be instantiated in the
+// translation unit that defines the variable.
+struct SymbolAddressCache {
+  struct Entry {
+    int device;
+    void* ctx;
+    void* addr;
+  };
+  std::mutex mu;
+  std::vector<Entry> entries;
+
+  template <typename T> dg_status get(const T& symbol, void** out) {
+    int dev = -1;
+    void* ctx = nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      set_last_error("no usable CUDA device");
+      return DG_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (current_context(&ctx))
+      for (const Entry& e : entries)
+        if (e.device == dev && e.ctx == ctx) {
+          *out = e.addr;
+          return DG_OK;
+        }
+    // not seen in this context (the lookup also makes the device's primary
+    // context current if no context was yet)
+    void* p = nullptr;
+    const cudaError_t err = cudaGetSymbolAddress(&p, symbol);
+    if (err != cudaSuccess || !p || !current_context(&ctx)) {
+      cudaGetLastError();
+      set_last_error(std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(err));
+      return DG_ERR_CUDA;
+    }
+    entries.push_back({dev, ctx, p});
+    *out = p;
+    return DG_OK;
+  }
+};
+
+// Device error word of the single-operation entry points (dg_ops.cu); the
+// allocation-free LM head has its own beside its scratch (dg_noalloc.cu).
+dg_status ops_error_word(int** out);
+dg_status noalloc_error_word(int** out);
+
 // Launch with programmatic stream serialization (see griddep_wait in
 // dg_common.cuh); the kernel must call griddep_wait() before using its
 // predecessors' outputs.
+// Programmatic launch is dropped (plain stream order) while this is set on
+// the launching thread: for graphs whose bodies take no programmatic edges.
+inline thread_local bool t_pdl_off = false;
+
 template <typename... KArgs, typename... Args>
 inline void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                        Args&&... args) {
@@ -65,7 +124,7 @@ inline void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = t_pdl_off ? 0 : 1;
   cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -162,12 +221,22 @@ struct CanvasState {
   uint8_t* done;
   int32_t* all_done;
   uint32_t* counters;  // [B + 1], zero between launches
+  int32_t* loop_iter;  // steps run by the current device-side decode loop
+};
+// A device-side decode loop: the conditional node that repeats the step, and
+// the most steps it may take (the loop ends once every canvas is done).
+struct DecodeLoop {
+  cudaGraphConditionalHandle handle = 0;
+  int cap = 0;
 };
 void launch_init_canvas(Exec& ex, const CanvasState& cs, int B, int C, int V);
 // Merge the LM-head partials into ent/am; with `sched` non-null also run the
 // freeze / stop / re-noise selection on every canvas.
+// With `loop` set, the step is the body of a device-side decode loop: the
+// kernel that finds every canvas done (or the cap reached) ends the loop.
 void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uint8_t* fmask,
-                         const CanvasState* cs, const dg_schedule* sched, int B, int C, int V);
+                         const CanvasState* cs, const dg_schedule* sched, int B, int C, int V,
+                         const DecodeLoop* loop = nullptr);
 
 }  // namespace dg
 
@@ -214,7 +283,13 @@ struct dg_ctx {
   std::vector<cudaGraphExec_t> graphs;
   dg_schedule graph_sched{};
   int graph_launches = 0;
-  std::vector<cudaEvent_t> ev_start, ev_stop;
-  cudaEvent_t cur_ev_start = nullptr, cur_ev_stop = nullptr;  // set while capturing
+  // timing event pairs per timed kernel (DG_KERNEL_LMHEAD, DG_KERNEL_ATTENTION)
+  std::vector<cudaEvent_t> ev_start[2], ev_stop[2];
+  cudaEvent_t cur_ev_start[2] = {nullptr, nullptr}, cur_ev_stop[2] = {nullptr, nullptr};  // set while capturing
+  // dg_decode_block's graph: the step as the body of a conditional while node
+  cudaGraphExec_t decode_graph = nullptr;
+  dg_schedule decode_sched{};
+  dg::DecodeLoop loop{};
+  const dg::DecodeLoop* cur_loop = nullptr;  // set while capturing the loop body
   long long step_launch_count = 0;
 };

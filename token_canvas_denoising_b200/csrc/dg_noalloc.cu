@@ -1,13 +1,12 @@
 // dg_lmhead_entropy_noalloc: the fused LM head + entropy/argmax without any
 // device allocation. Some callers cannot allocate device memory at the point
-// where they need this operation: code that is being recorded into a CUDA
-// graph (an allocation cannot be part of the recorded work), and applications
-// whose device memory is fully reserved up front by their own allocator, where
-// a driver allocation in the middle of a step would fail or fragment memory.
-// For them the per-CTA partial results that dg_lmhead_entropy keeps in a
-// temporary buffer live in a fixed, library-owned device array instead.
-#include <mutex>
-
+// where they need this operation: applications whose device memory is fully
+// reserved up front by their own allocator, where a driver allocation in the
+// middle of a step fails or fragments what is left; and hosts that give a
+// plug-in only the buffers they pass it and forbid it to allocate (or to pay
+// the device-wide synchronisation an allocation can cost). For them the
+// per-CTA partial results that dg_lmhead_entropy keeps in a temporary buffer
+// live in a fixed, library-owned device array instead.
 #include "dg_internal.cuh"
 #include "dg_ops.h"
 
@@ -18,37 +17,25 @@ namespace {
 // until the process exits, and every call on that GPU shares it.
 constexpr size_t kScratchRecords = 65536;
 static __device__ __align__(256) dg::LmRec g_lm_scratch[kScratchRecords];
+// Device error word of this entry point's kernels (a bounded wait that gave
+// up, a NaN entropy), read and cleared by dg_ops_check.
+static __device__ int g_noalloc_err;
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-dg::LmRec* g_scratch_ptr[kMaxDevices] = {nullptr};
-
-// The device address of the scratch array on the current device. The array's
-// name in host code is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
-dg_status scratch_for_current_device(dg::LmRec** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    dg::set_last_error("no usable CUDA device");
-    return DG_ERR_CUDA;
-  }
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_lm_scratch);
-    if (e != cudaSuccess || !p) {
-      cudaGetLastError();
-      dg::set_last_error(std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(e));
-      return DG_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = static_cast<dg::LmRec*>(p);
-  }
-  *out = g_scratch_ptr[dev];
-  return DG_OK;
-}
+// In host code the names above are host-side stand-ins, not device
+// addresses: the addresses are looked up per device and context (the first
+// call on each device does it) and passed to the kernels.
+dg::SymbolAddressCache g_scratch_addr, g_err_addr;
 
 }  // namespace
+
+namespace dg {
+dg_status noalloc_error_word(int** out) {
+  void* p = nullptr;
+  const dg_status st = g_err_addr.get(g_noalloc_err, &p);
+  *out = static_cast<int*>(p);
+  return st;
+}
+}  // namespace dg
 
 extern "C" {
 
@@ -68,14 +55,15 @@ dg_status dg_lmhead_entropy_noalloc(int32_t dtype, const void* hs, const void* l
     dg::set_last_error("unsupported: d % 8 (bf16: d % 64 and V % 256)");
     return DG_ERR_UNSUPPORTED;
   }
-  dg::LmRec* scratch = nullptr;
-  dg_status st = scratch_for_current_device(&scratch);
-  if (st != DG_OK) return st;
   dg::Exec ex;
   ex.stream = static_cast<cudaStream_t>(stream);
   int dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&ex.sm_count, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ex.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    dg::set_last_error("no usable CUDA device");
+    return DG_ERR_CUDA;
+  }
   dg::LmPartials part;
   part.P = dtype == DG_BF16 ? dg::lmhead_tc_partitions(M, V, ex.sm_count) : std::max(1, std::min(128, V / 1024));
   if ((size_t)M * (size_t)part.P > kScratchRecords) {
@@ -83,7 +71,13 @@ dg_status dg_lmhead_entropy_noalloc(int32_t dtype, const void* hs, const void* l
                        " exceeds the fixed scratch of " + std::to_string(kScratchRecords) + " records");
     return DG_ERR_UNSUPPORTED;
   }
-  part.rec = scratch;  // every record the merge reads is written by this call's LM-head kernel
+  void* scratch = nullptr;
+  dg_status st = g_scratch_addr.get(g_lm_scratch, &scratch);
+  if (st == DG_OK) st = dg::noalloc_error_word(&ex.err);
+  if (st != DG_OK) return st;
+  // every record the merge reads is written by this call's LM-head kernel, so
+  // nothing left in the array by an earlier call is read
+  part.rec = static_cast<dg::LmRec*>(scratch);
   if (dtype == DG_BF16) {
     CUtensorMap a, b;
     if (!dg::lmhead_tc_prepare(hs, lm_head, M, d, V, &a, &b)) return DG_ERR_CUDA;

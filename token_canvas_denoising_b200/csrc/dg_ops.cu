@@ -33,16 +33,34 @@ dg_status cuda_status(cudaError_t e, const char* what) {
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-dg::Exec make_exec(void* stream) {
-  dg::Exec ex;
-  ex.stream = static_cast<cudaStream_t>(stream);
+// Device error word of these entry points: their kernels record the first
+// device-side failure here (a bounded wait that gave up, a NaN entropy) and
+// dg_ops_check reads and clears it.
+static __device__ int g_ops_err;
+dg::SymbolAddressCache g_ops_err_addr;
+
+dg_status make_exec(void* stream, dg::Exec* ex) {
+  ex->stream = static_cast<cudaStream_t>(stream);
   int dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&ex.sm_count, cudaDevAttrMultiProcessorCount, dev);
-  return ex;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ex->sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    set_last_error("no usable CUDA device");
+    return DG_ERR_CUDA;
+  }
+  return dg::ops_error_word(&ex->err);
 }
 
 }  // namespace
+
+namespace dg {
+dg_status ops_error_word(int** out) {
+  void* p = nullptr;
+  const dg_status st = g_ops_err_addr.get(g_ops_err, &p);
+  *out = static_cast<int*>(p);
+  return st;
+}
+}  // namespace dg
 
 extern "C" {
 
@@ -54,7 +72,8 @@ dg_status dg_lmhead_entropy(int32_t dtype, const void* hs, const void* lm_head, 
   OP_ARG(al16(hs) && al16(lm_head), "hs / lm_head must be 16-byte aligned");
   OP_UNSUP(d % 8 == 0, "d % 8 != 0");
   if (dtype == DG_BF16) OP_UNSUP(d % 64 == 0 && V % 256 == 0, "bf16 needs d % 64 == 0 and V % 256 == 0");
-  dg::Exec ex = make_exec(stream);
+  dg::Exec ex;
+  if (dg_status est = make_exec(stream, &ex)) return est;
   dg::LmPartials part;
   part.P = dtype == DG_BF16 ? dg::lmhead_tc_partitions(M, V, ex.sm_count) : std::max(1, std::min(128, V / 1024));
   dg_status st = cuda_status(cudaMallocAsync((void**)&part.rec, sizeof(dg::LmRec) * (size_t)M * part.P, ex.stream),
@@ -90,7 +109,8 @@ dg_status dg_attention(int32_t dtype, const void* q, const void* kc, const void*
     if (prefix_len[b] > 0) OP_ARG(prefix_k && prefix_v && prefix_k[b] && prefix_v[b], "NULL prefix pointer");
     pd[b] = {prefix_len[b] ? prefix_k[b] : nullptr, prefix_len[b] ? prefix_v[b] : nullptr, prefix_len[b], 0};
   }
-  dg::Exec ex = make_exec(stream);
+  dg::Exec ex;
+  if (dg_status est = make_exec(stream, &ex)) return est;
   if (dtype == DG_BF16) {
     OP_ARG(al16(q) && al16(kc) && al16(vc) && al16(o), "buffers must be 16-byte aligned");
     dg::AttnShape sh{B, C, Hq, Hk, h};
@@ -128,12 +148,33 @@ dg_status dg_attention(int32_t dtype, const void* q, const void* kc, const void*
   return st;
 }
 
+dg_status dg_ops_check(void* stream) {
+  int* words[2] = {nullptr, nullptr};
+  dg_status st = dg::ops_error_word(&words[0]);
+  if (st == DG_OK) st = dg::noalloc_error_word(&words[1]);
+  if (st != DG_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h[2] = {0, 0};
+  for (int i = 0; i < 2; ++i) {
+    st = cuda_status(cudaMemcpyAsync(&h[i], words[i], sizeof(int), cudaMemcpyDeviceToHost, s), "cudaMemcpyAsync");
+    if (st == DG_OK) st = cuda_status(cudaMemsetAsync(words[i], 0, sizeof(int), s), "cudaMemsetAsync");
+    if (st != DG_OK) return st;
+  }
+  st = cuda_status(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  if (st != DG_OK) return st;
+  const int code = h[0] ? h[0] : h[1];
+  if (code == 0) return DG_OK;
+  set_last_error("device-side check failed in a single-operation call (code " + std::to_string(code) + ")");
+  return code == dg::kDevWaitTimeout ? DG_ERR_TIMEOUT : DG_ERR_DEVICE_CHECK;
+}
+
 dg_status dg_linear(int32_t dtype, const void* a, const void* w, const void* residual, void* out, int32_t M,
                     int32_t N, int32_t K, void* stream) {
   OP_ARG(dtype == DG_F32 || dtype == DG_BF16, "dtype");
   OP_ARG(a && w && out, "NULL buffer");
   OP_ARG(M >= 1 && N >= 1 && K >= 1, "sizes");
-  dg::Exec ex = make_exec(stream);
+  dg::Exec ex;
+  if (dg_status est = make_exec(stream, &ex)) return est;
   if (dtype == DG_BF16) {
     OP_UNSUP(K % 64 == 0 && N % 64 == 0, "bf16 needs K % 64 == 0 and N % 64 == 0");
     OP_ARG(al16(a) && al16(w) && al16(out) && (!residual || al16(residual)), "buffers must be 16-byte aligned");

@@ -45,6 +45,9 @@ struct SelectArgs {
   uint8_t* done;
   int32_t* all_done;
   uint32_t* counters;   // [B + 1], zero on entry, left zero
+  int32_t* loop_iter;   // steps of the device-side decode loop (with cond)
+  cudaGraphConditionalHandle cond;  // 0, or the decode loop's condition
+  int loop_cap;
   int32_t* err;
   int B, C, V, max_steps, adaptive;
   float stop_entropy;
@@ -192,12 +195,19 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
       for (int i = 0; i < a.B; ++i) all &= (__ldcg(&a.done[i]) != 0) ? 1 : 0;
       *a.all_done = all;
       a.counters[a.B] = 0;
+      if (a.cond) {  // the step is the body of a device-side decode loop
+        const int it = *a.loop_iter + 1;
+        *a.loop_iter = it;
+        if (!all && it >= a.loop_cap) set_error(a.err, kDevLoopCap);
+        cudaGraphSetConditional(a.cond, (!all && it < a.loop_cap) ? 1u : 0u);
+      }
     }
   }
 }
 
 void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uint8_t* fmask,
-                         const CanvasState* cs, const dg_schedule* sched, int B, int C, int V) {
+                         const CanvasState* cs, const dg_schedule* sched, int B, int C, int V,
+                         const DecodeLoop* loop) {
   SelectArgs a{};
   a.part = part;
   a.ent = ent;
@@ -219,6 +229,11 @@ void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uin
     a.max_steps = sched->max_steps;
     a.adaptive = sched->adaptive_stop;
     a.stop_entropy = sched->stop_entropy;
+    a.loop_iter = cs->loop_iter;
+    if (loop) {
+      a.cond = loop->handle;
+      a.loop_cap = loop->cap;
+    }
   }
   dim3 grid(ceil_div(C, 8), B);
   launch_pdl(merge_select_kernel, grid, dim3(256), 0, ex.stream, a);

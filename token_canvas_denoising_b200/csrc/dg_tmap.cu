@@ -47,4 +47,19 @@ bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64
   return true;
 }
 
+bool current_context(void** ctx) {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  }
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS || !c) return false;
+  *ctx = c;
+  return true;
+}
+
 }  // namespace dg

@@ -43,7 +43,7 @@ import math
 
 import numpy as np
 
-from .numerics import round_storage, widen
+from .numerics import e4m3_to_f64, quantize_rows_e4m3, round_storage, widen
 from .philox import canvas_draw
 
 LM_CHUNK = 8192  # vocab rows widened to fp64 at a time (memory only)
@@ -210,7 +210,17 @@ def moe_block(model, Hs, choice=None):
 
 
 def lm_head_logits(model, Hs_rows):
-    """Unscaled logits Hs W_lm^T in fp64 for the given rows: [rows, V]."""
+    """Unscaled logits Hs W_lm^T in fp64 for the given rows: [rows, V].
+
+    With FP8 LM-head weights (model["lm_head_e4m3"]: e4m3 codes [V][d] with
+    power-of-two row scales 2^model["lm_head_exp"][v]) the product is the FP8
+    one: each row of Hs is quantized to e4m3 with its own power-of-two scale
+    2^e_r, and x[r][v] = 2^(e_r + e_v) sum_k q_r[k] q_v[k]. Every e4m3 value is
+    an integer multiple of 2^-9 of magnitude below 2^9, so each product has at
+    most 8 significant bits and a sum over d <= 2^20 terms stays an exact
+    multiple of 2^-18 below 2^38: the fp64 dot product is exact."""
+    if model.get("lm_head_e4m3") is not None:
+        return lm_head_logits_e4m3(model, Hs_rows)
     dt = model["dtype"]
     W = model["lm_head"]
     V = W.shape[0]
@@ -218,6 +228,21 @@ def lm_head_logits(model, Hs_rows):
     for v0 in range(0, V, LM_CHUNK):
         v1 = min(V, v0 + LM_CHUNK)
         out[:, v0:v1] = Hs_rows @ widen(W[v0:v1], dt).T
+    return out
+
+
+def lm_head_logits_e4m3(model, Hs_rows):
+    """The FP8 LM head (see lm_head_logits)."""
+    qa, ea = quantize_rows_e4m3(Hs_rows)
+    a = e4m3_to_f64(qa)
+    W = model["lm_head_e4m3"]
+    ew = np.asarray(model["lm_head_exp"], dtype=np.int64)
+    V = W.shape[0]
+    out = np.empty((Hs_rows.shape[0], V), dtype=np.float64)
+    for v0 in range(0, V, LM_CHUNK):
+        v1 = min(V, v0 + LM_CHUNK)
+        dot = a @ e4m3_to_f64(W[v0:v1]).T
+        out[:, v0:v1] = dot * np.exp2((ea[:, None] + ew[None, v0:v1]).astype(np.float64))
     return out
 
 

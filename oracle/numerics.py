@@ -54,3 +54,65 @@ def widen(w, dtype):
     if dtype == "bf16":
         return bf16_bits_to_f64(w)
     return np.asarray(w, dtype=np.float64)
+
+
+# ---------------------------------------------------------------- FP8 (e4m3)
+# The FP8 deployment the pages report ("DiffusionGemma深度拆解" 性能数据: H100
+# FP8; "谷歌DiffusionGemma" 引入扩散机制: the vLLM FP8 benchmark) stores the
+# LM-head weights in 8-bit floating point. e4m3 ("fn" variant): 1 sign bit, 4
+# exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
+# subnormals m/8 * 2^-6; S.1111.111 is NaN; no infinities; largest finite
+# 448 = 1.75 * 2^8.
+E4M3_MAX = 448.0
+
+
+def e4m3_to_f64(codes):
+    """e4m3 byte codes -> float64 (exact)."""
+    b = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((b & 0x80) != 0, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & (b & 7 == 7), np.nan, mag)
+    return sign * mag
+
+
+_E4M3_NONNEG = e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))  # codes 0..126, increasing
+
+
+def round_to_e4m3(x):
+    """float64 -> e4m3 byte codes, round to nearest with ties to the even code
+    (the even mantissa). |x| must not exceed 448: callers scale into range, so
+    no saturation rule is needed. The sign bit follows x (a negative value
+    that rounds to zero gives the code of -0)."""
+    x = np.asarray(x, dtype=np.float64)
+    if not np.all(np.abs(x) <= E4M3_MAX):
+        raise ValueError("value outside the e4m3 range")
+    a = np.abs(x)
+    hi = np.minimum(np.searchsorted(_E4M3_NONNEG, a, side="left"), 126)  # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - _E4M3_NONNEG[lo]
+    dhi = _E4M3_NONNEG[hi] - a
+    pick = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(dhi == 0, hi, pick)
+    return (pick.astype(np.uint8) | np.where(np.signbit(x), 0x80, 0).astype(np.uint8)).astype(np.uint8)
+
+
+def e4m3_scale_exponent(amax):
+    """The smallest integer e with 448 * 2^e >= amax (0 for amax = 0): the
+    power-of-two scale that brings a row's largest magnitude into the e4m3
+    range. With amax = f 2^k (f in [0.5, 1)) and 448 = 0.875 2^9 this is
+    k - 9 when f <= 0.875, else k - 8 (exact integer arithmetic)."""
+    amax = np.asarray(amax, dtype=np.float64)
+    f, k = np.frexp(amax)
+    e = np.where(f <= 0.875, k - 9, k - 8)
+    return np.where(amax > 0, e, 0).astype(np.int64)
+
+
+def quantize_rows_e4m3(x):
+    """Each row of x as e4m3 codes times a power of two: e = the row's
+    e4m3_scale_exponent, codes = round_to_e4m3(x * 2^-e) (the scaling is
+    exact). Returns (codes [rows][n], e [rows])."""
+    x = np.asarray(x, dtype=np.float64)
+    e = e4m3_scale_exponent(np.max(np.abs(x), axis=-1))
+    return round_to_e4m3(x * np.exp2(-e.astype(np.float64))[..., None]), e

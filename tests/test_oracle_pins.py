@@ -607,3 +607,81 @@ def test_planted_renoise_step_is_caught(monkeypatch):
     monkeypatch.setattr(om, "canvas_draw", lambda s, t, p, b, V: orig(s, t + 1, p, b, V))
     with pytest.raises(AssertionError):
         test_whole_loop_small_vocab(4, 5)
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) LM head
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    a = on.e4m3_to_f64(codes)
+    b = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(a), np.isnan(b)) and np.isnan(a).sum() == 2
+    assert np.array_equal(a[~np.isnan(a)], b[~np.isnan(b)])
+    assert np.nanmax(a) == 448.0 and a[1] == 2.0 ** -9
+
+
+def test_e4m3_rounding_matches_torch_cast():
+    """Round to nearest, ties to even, against torch's float8_e4m3fn cast:
+    random values over the whole range and every midpoint between adjacent
+    values (the ties), including the subnormal range and both signs."""
+    rng = np.random.default_rng(5)
+    vals = on.e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))
+    mids = 0.5 * (vals[1:] + vals[:-1])
+    x = np.concatenate([rng.uniform(-448, 448, 20000), np.exp2(rng.uniform(-12, 8.8, 20000)) *
+                        rng.choice([-1, 1], 20000), mids, -mids, vals, -vals])
+    x = np.clip(x, -448, 448)
+    got = on.round_to_e4m3(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_scale_exponent_is_the_smallest_that_fits():
+    rng = np.random.default_rng(6)
+    amax = np.concatenate([np.exp2(rng.uniform(-20, 20, 5000)), 448.0 * np.exp2(np.arange(-10, 10.0)),
+                           448.0 * np.exp2(np.arange(-10, 10.0)) * (1 + 2.0 ** -20), [1.0, 3.0, 449.0]])
+    e = on.e4m3_scale_exponent(amax)
+    assert np.all(448.0 * np.exp2(e.astype(float)) >= amax)
+    assert np.all(448.0 * np.exp2(e.astype(float) - 1) < amax)
+    assert on.e4m3_scale_exponent(np.array([0.0]))[0] == 0
+
+
+def test_e4m3_dot_products_are_exact_in_fp64():
+    """Every e4m3 value is n 2^-9 with an integer n, so a dot product of two
+    code rows is 2^-18 times an integer sum: the fp64 matmul equals it exactly."""
+    rng = np.random.default_rng(7)
+    a = rng.integers(0, 256, (3, 2816), dtype=np.uint8)
+    w = rng.integers(0, 256, (5, 2816), dtype=np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0  # no NaN codes
+    w[(w & 0x7F) == 0x7F] = 0
+    fa, fw = on.e4m3_to_f64(a), on.e4m3_to_f64(w)
+    got = fa @ fw.T
+    na = [[int(round(v * 512)) for v in row] for row in fa]
+    nw = [[int(round(v * 512)) for v in row] for row in fw]
+    for i in range(3):
+        for j in range(5):
+            assert got[i, j] == sum(x * y for x, y in zip(na[i], nw[j])) * 2.0 ** -18
+
+
+def test_fp8_lm_head_logits_worked_by_hand():
+    """Hs row (1, 0.3): largest magnitude 1 -> scale 2^-8 (448 2^-8 = 1.75 >= 1,
+    0.875 < 1); 0.3 * 2^8 = 76.8 lies between the e4m3 values 72 and 80 and
+    rounds to 80, i.e. 0.3125. With weight rows (1, 1), (2, -4) at scale 2^0
+    and (1.5, 1) at 2^-1 the logits are 1.3125, 0.75, 0.90625.
+    Hs row (1, 3 2^-17): the small entry scales to 3 2^-9, the e4m3 subnormal
+    with mantissa 3, exactly; through the weight row (0, 1) the logit is
+    3 2^-17 (a scale twice as large would give 1.5 2^-9, a tie that rounds
+    to 2 2^-9, and the logit 4 2^-17)."""
+    w = np.array([[1.0, 1.0], [2.0, -4.0], [1.5, 1.0], [0.0, 1.0]])
+    m = {"dtype": "bf16", "lm_head_e4m3": on.round_to_e4m3(w), "lm_head_exp": np.array([0, 0, -1, 0])}
+    got = om.lm_head_logits(m, np.array([[1.0, 0.3], [1.0, 3 * 2.0 ** -17]]))
+    assert got[0].tolist() == [1.3125, 2.0 - 4 * 0.3125, 0.5 * (1.5 + 0.3125), 0.3125]
+    assert got[0, 2] == 0.90625
+    assert got[1, 3] == 3 * 2.0 ** -17
+
+
+def test_planted_fp8_scale_off_by_one_is_caught(monkeypatch):
+    real = on.e4m3_scale_exponent
+    monkeypatch.setattr(on, "e4m3_scale_exponent", lambda amax: real(amax) + 1)
+    with pytest.raises(AssertionError):
+        test_fp8_lm_head_logits_worked_by_hand()
+    with pytest.raises(AssertionError):
+        test_e4m3_scale_exponent_is_the_smallest_that_fits()

@@ -65,6 +65,35 @@ def prewiden(model, keys=("wq", "wk", "wv", "wo", "lm_head")):
     return m
 
 
+def n_layers(model):
+    """Number of attention layers. A model dict with "n_layers" holds its
+    layer weights stacked layer-major (wq, wk, wv, wo as [L][out][in]) and its
+    prompt caches as [L][S][Hk][h] per request; without it the model has one
+    layer and unstacked arrays."""
+    return int(model.get("n_layers", 1))
+
+
+def layer(model, l):
+    """The one-layer view of layer l: its own wq, wk, wv, wo."""
+    if "n_layers" not in model:
+        assert l == 0
+        return model
+    m = dict(model)
+    for k in ("wq", "wk", "wv", "wo"):
+        m[k] = model[k][l]
+    return m
+
+
+def layer_prefix(model, prefix, l):
+    """Each request's prompt K/V of layer l."""
+    if "n_layers" not in model:
+        assert l == 0
+        return prefix
+    _, _, Hk, h, _ = dims(model)
+    return [(np.asarray(k).reshape(n_layers(model), -1, Hk, h)[l], np.asarray(v).reshape(n_layers(model), -1, Hk, h)[l])
+            for k, v in prefix]
+
+
 def kv_head_of(q, Hq, Hk):
     """Consecutive query heads share one KV head."""
     return q // (Hq // Hk)
@@ -98,6 +127,7 @@ def block_kv(model, tok):
     K/V depend only on its own embedding, so that pass is the K/V projection of
     the committed tokens. tok: [B][C]; returns K, V as [B][C][Hk][h] (fp64
     values rounded to the storage dtype)."""
+    assert n_layers(model) == 1, "block K/V are defined for the single-layer model"
     B, C = np.asarray(tok).shape
     _, Kc, Vc = project_qkv(model, embed(model, tok))
     _, _, Hk, h, _ = dims(model)
@@ -213,9 +243,9 @@ def lm_head_logits(model, Hs_rows):
     """Unscaled logits Hs W_lm^T in fp64 for the given rows: [rows, V].
 
     With FP8 LM-head weights (model["lm_head_e4m3"]: e4m3 codes [V][d] with
-    power-of-two row scales 2^model["lm_head_exp"][v]) the product is the FP8
-    one: each row of Hs is quantized to e4m3 with its own power-of-two scale
-    2^e_r, and x[r][v] = 2^(e_r + e_v) sum_k q_r[k] q_v[k]. Every e4m3 value is
+    power-of-two row scales s_v = model["lm_head_scale"][v]) the product is the
+    FP8 one: each row of Hs is quantized to e4m3 with its own power-of-two
+    scale 2^e_r, and x[r][v] = 2^e_r s_v sum_k q_r[k] q_v[k]. Every e4m3 value is
     an integer multiple of 2^-9 of magnitude below 2^9, so each product has at
     most 8 significant bits and a sum over d <= 2^20 terms stays an exact
     multiple of 2^-18 below 2^38: the fp64 dot product is exact."""
@@ -236,13 +266,13 @@ def lm_head_logits_e4m3(model, Hs_rows):
     qa, ea = quantize_rows_e4m3(Hs_rows)
     a = e4m3_to_f64(qa)
     W = model["lm_head_e4m3"]
-    ew = np.asarray(model["lm_head_exp"], dtype=np.int64)
+    sw = np.asarray(model["lm_head_scale"], dtype=np.float64)
     V = W.shape[0]
     out = np.empty((Hs_rows.shape[0], V), dtype=np.float64)
     for v0 in range(0, V, LM_CHUNK):
         v1 = min(V, v0 + LM_CHUNK)
         dot = a @ e4m3_to_f64(W[v0:v1]).T
-        out[:, v0:v1] = dot * np.exp2((ea[:, None] + ew[None, v0:v1]).astype(np.float64))
+        out[:, v0:v1] = dot * np.exp2(ea.astype(np.float64))[:, None] * sw[None, v0:v1]
     return out
 
 
@@ -331,15 +361,32 @@ def copy_state(st):
     return {k: v.copy() for k, v in st.items()}
 
 
+def attention_layer(model, prefix, X, B, C, l):
+    """Layer l: Q/K/V of its input X, attention over the layer's prompt K/V
+    and the canvas, Wo + residual. Returns (Q, Kc, Vc, O, output)."""
+    ml, pl = layer(model, l), layer_prefix(model, prefix, l)
+    Q, Kc, Vc = project_qkv(ml, X)
+    O = attention(ml, Q, Kc, Vc, pl, B, C)
+    return Q, Kc, Vc, O, out_proj_residual(ml, X, O)
+
+
 def forward(model, prefix, tok, inv_temp):
-    """One forward pass over all canvases: returns (ent, am, gap, extras)."""
+    """One forward pass over all canvases: returns (ent, am, gap, extras).
+
+    Layers in sequence, each fed the previous one's output (the residual
+    stream); the LM head reads the last layer's output. extras holds the
+    embedding X, the last layer's Q, canvas K/V and attention output O, every
+    layer's output ("layers") and Hs_attn (the last one)."""
     B, C = tok.shape
     X = embed(model, tok)
-    Q, Kc, Vc = project_qkv(model, X)
-    O = attention(model, Q, Kc, Vc, prefix, B, C)
-    Hs = out_proj_residual(model, X, O)
-    extras = {"X": X, "Q": Q, "Kc": Kc, "Vc": Vc, "O": O, "Hs_attn": Hs}
+    extras = {"X": X, "layers": []}
+    Hs = X
+    for l in range(n_layers(model)):
+        Q, Kc, Vc, O, Hs = attention_layer(model, prefix, Hs, B, C, l)
+        extras["layers"].append(Hs)
+    extras.update({"Q": Q, "Kc": Kc, "Vc": Vc, "O": O, "Hs_attn": Hs})
     if model.get("n_experts", 0):
+        assert n_layers(model) == 1, "the MoE block is defined for the single-layer model"
         Hs, route = moe_block(model, Hs)
         extras["route"] = route
     extras["Hs"] = Hs

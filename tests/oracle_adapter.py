@@ -7,8 +7,13 @@ from oracle import model as om
 def oracle_model(wl):
     c = wl.cfg
     m = {"dtype": c.dtype, "d": c.d, "Hq": c.Hq, "Hk": c.Hk, "h": c.h, "V": c.V}
+    if c.n_layers:  # stacked layer weights and per-layer prompt caches
+        m["n_layers"] = c.n_layers
     for k in ("embed", "wq", "wk", "wv", "wo", "lm_head"):
         m[k] = wl.weights[k]
+    if c.lm_fp8:  # e4m3 codes with power-of-two row scales
+        m["lm_head_e4m3"] = wl.weights["lm_head"]
+        m["lm_head_scale"] = wl.weights["lm_head_scale"]
     if c.n_experts:
         m.update(n_experts=c.n_experts, top_k=c.top_k, moe_inter=c.moe_inter,
                  n_shared=c.n_shared)

@@ -671,7 +671,7 @@ def test_fp8_lm_head_logits_worked_by_hand():
     3 2^-17 (a scale twice as large would give 1.5 2^-9, a tie that rounds
     to 2 2^-9, and the logit 4 2^-17)."""
     w = np.array([[1.0, 1.0], [2.0, -4.0], [1.5, 1.0], [0.0, 1.0]])
-    m = {"dtype": "bf16", "lm_head_e4m3": on.round_to_e4m3(w), "lm_head_exp": np.array([0, 0, -1, 0])}
+    m = {"dtype": "bf16", "lm_head_e4m3": on.round_to_e4m3(w), "lm_head_scale": np.array([1.0, 1.0, 0.5, 1.0])}
     got = om.lm_head_logits(m, np.array([[1.0, 0.3], [1.0, 3 * 2.0 ** -17]]))
     assert got[0].tolist() == [1.3125, 2.0 - 4 * 0.3125, 0.5 * (1.5 + 0.3125), 0.3125]
     assert got[0, 2] == 0.90625
@@ -685,3 +685,40 @@ def test_planted_fp8_scale_off_by_one_is_caught(monkeypatch):
         test_fp8_lm_head_logits_worked_by_hand()
     with pytest.raises(AssertionError):
         test_e4m3_scale_exponent_is_the_smallest_that_fits()
+
+
+# ---------------------------------------------------------------- layer stack
+def _layers_cfg(L, **kw):
+    return fx.Config(name="layers", B=2, C=6, S=(5, 0), d=16, Hq=2, Hk=1, h=8, V=32, dtype="f32", max_steps=4,
+                     weight_seed=61, canvas_seeds=(1, 2), n_layers=L, **kw)
+
+
+def test_one_stacked_layer_equals_the_single_layer_model():
+    st = None
+    outs = []
+    for L in (0, 1):
+        wl = fx.make_workload(_layers_cfg(L))
+        m, pre = oracle_model(wl), oracle_prefix(wl)
+        st = om.init_state(wl.seeds, 6, 32) if st is None else st
+        outs.append(om.forward(m, pre, st["tok"], None))
+    for a, b in zip(outs[0][:3], outs[1][:3]):
+        assert np.array_equal(a, b)
+
+
+def test_second_layer_with_zero_output_projection_is_the_identity():
+    """With Wo = 0 in layer 2 its output equals its input, so the two-layer
+    model's entropies equal those of layer 1 alone."""
+    wl2 = fx.make_workload(_layers_cfg(2))
+    m2, pre2 = oracle_model(wl2), oracle_prefix(wl2)
+    m2["wo"] = m2["wo"].copy()
+    m2["wo"][1] = 0
+    m1 = dict(m2, n_layers=1, wq=m2["wq"][:1], wk=m2["wk"][:1], wv=m2["wv"][:1], wo=m2["wo"][:1])
+    pre1 = [(k[:1], v[:1]) for k, v in pre2]
+    st = om.init_state(wl2.seeds, 6, 32)
+    e2, a2, _, x2 = om.forward(m2, pre2, st["tok"], None)
+    e1, a1, _, x1 = om.forward(m1, pre1, st["tok"], None)
+    assert np.array_equal(x2["layers"][1], x2["layers"][0])
+    assert np.array_equal(e1, e2) and np.array_equal(a1, a2)
+    # and a non-zero second layer changes them
+    e3, *_ = om.forward(oracle_model(wl2), pre2, st["tok"], None)
+    assert not np.allclose(e3, e1)

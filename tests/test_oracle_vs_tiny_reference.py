@@ -49,3 +49,14 @@ def test_random_small_cases(V, C, B, adaptive):
     cfg = fx.Config(name="tinyr", B=B, C=C, S=tuple(2 + 3 * b for b in range(B)), d=8, Hq=2, Hk=1, h=4, V=V,
                     dtype="f32", max_steps=5, weight_seed=20 + V + C, canvas_seeds=tuple(30 + b for b in range(B)))
     _compare(cfg, adaptive)
+
+
+@pytest.mark.parametrize("L,V,C,B,adaptive", [(2, 8, 6, 2, False), (3, 4, 5, 1, True), (2, 8, 4, 2, True)])
+def test_multi_layer_small_cases(L, V, C, B, adaptive):
+    """A stack of L layers (each attention + Wo + residual over its own prompt
+    K/V, fed the previous layer's output) decodes identically in both
+    implementations."""
+    cfg = fx.Config(name="tinyl", B=B, C=C, S=tuple(2 + 3 * b for b in range(B)), d=8, Hq=2, Hk=1, h=4, V=V,
+                    dtype="f32", max_steps=5, weight_seed=40 + L + V, canvas_seeds=tuple(50 + b for b in range(B)),
+                    n_layers=L)
+    _compare(cfg, adaptive)

@@ -39,28 +39,31 @@ def _rows(a):
 
 
 def forward_canvas(w, Kp, Vp, tok, Hq, Hk, h):
-    """Entropy and argmax of every position of one canvas."""
-    E, Wq, Wk, Wv, Wo, Wl = w
+    """Entropy and argmax of every position of one canvas. w = (E, layers, Wl)
+    with layers a list of (Wq, Wk, Wv, Wo); Kp, Vp: per layer, the prompt
+    keys / values (lists of rows)."""
+    E, layers, Wl = w
     d = len(E[0])
     X = [E[t] for t in tok]
     proj = lambda W, x: [f32(sum(x[k] * W[j][k] for k in range(d))) for j in range(len(W))]
-    Q = [proj(Wq, x) for x in X]
-    K = Kp + [proj(Wk, x) for x in X]
-    Vv = Vp + [proj(Wv, x) for x in X]
-    O = []
-    for q in Q:
-        o = []
-        for hq in range(Hq):
-            g = hq // (Hq // Hk)
-            s = [sum(q[hq * h + i] * k[g * h + i] for i in range(h)) / math.sqrt(h) for k in K]
-            m = max(s)
-            e = [math.exp(v - m) for v in s]
-            z = sum(e)
-            o += [f32(sum(e[j] / z * Vv[j][g * h + i] for j in range(len(K)))) for i in range(h)]
-        O.append(o)
+    for (Wq, Wk, Wv, Wo), kp, vp in zip(layers, Kp, Vp):
+        Q = [proj(Wq, x) for x in X]
+        K = kp + [proj(Wk, x) for x in X]
+        Vv = vp + [proj(Wv, x) for x in X]
+        O = []
+        for q in Q:
+            o = []
+            for hq in range(Hq):
+                g = hq // (Hq // Hk)
+                s = [sum(q[hq * h + i] * k[g * h + i] for i in range(h)) / math.sqrt(h) for k in K]
+                m = max(s)
+                e = [math.exp(v - m) for v in s]
+                z = sum(e)
+                o += [f32(sum(e[j] / z * Vv[j][g * h + i] for j in range(len(K)))) for i in range(h)]
+            O.append(o)
+        X = [[f32(x[k] + sum(o[j] * Wo[k][j] for j in range(len(o)))) for k in range(d)] for x, o in zip(X, O)]
     ents, ams = [], []
-    for x, o in zip(X, O):
-        hs = [f32(x[k] + sum(o[j] * Wo[k][j] for j in range(len(o)))) for k in range(d)]
+    for hs in X:
         lg = [sum(hs[k] * wl[k] for k in range(d)) for wl in Wl]
         m = max(lg)
         e = [math.exp(v - m) for v in lg]
@@ -73,11 +76,16 @@ def forward_canvas(w, Kp, Vp, tok, Hq, Hk, h):
 def decode(weights, prefix, seeds, C, V, Hq, Hk, h, T, stop_entropy, adaptive, init_tok=None):
     """Whole decode of every canvas; returns (tokens [B][C], steps [B],
     entropies [B][steps][C])."""
-    w = [_rows(weights[k]) for k in ("embed", "wq", "wk", "wv", "wo", "lm_head")]
+    stacked = np.asarray(weights["wq"]).ndim == 3  # [L][out][in] per layer
+    L = np.asarray(weights["wq"]).shape[0] if stacked else 1
+    per_layer = lambda k: [weights[k][l] for l in range(L)] if stacked else [weights[k]]
+    layers = list(zip(*[[_rows(m) for m in per_layer(k)] for k in ("wq", "wk", "wv", "wo")]))
+    w = (_rows(weights["embed"]), layers, _rows(weights["lm_head"]))
     out_tok, out_steps, out_ent = [], [], []
     for b, seed in enumerate(seeds):
-        Kp = [list(map(float, np.asarray(r, np.float64).reshape(-1))) for r in prefix[b][0]]
-        Vp = [list(map(float, np.asarray(r, np.float64).reshape(-1))) for r in prefix[b][1]]
+        rows = lambda a: [[list(map(float, np.asarray(r, np.float64).reshape(-1))) for r in lay]
+                          for lay in (np.asarray(a).reshape(L, -1, Hk, h))]
+        Kp, Vp = rows(prefix[b][0]), rows(prefix[b][1])
         tok = [draw(seed, 0, p, b, V) for p in range(C)] if init_tok is None else list(init_tok[b])
         frozen = [False] * C
         t = 0

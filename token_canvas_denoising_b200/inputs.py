@@ -13,6 +13,8 @@ Workloads follow the five synthetic configurations of the method's hot path
   vocab262k  B1 C256 S4096   d2816 Hq16/Hk8 h128 V262144  bf16  T=48, invT log-uniform [1/5, 1/0.05]
   longctx    B4 C256 S32768  d2816 Hq16/Hk8 h128 V262144  bf16  T=48, prefix scale U[0.5, 2] per (request, head)
   moe        vocab262k + MoE 128 experts + 1 shared, top-8, GeGLU intermediate 704
+  *_fp8      vocab262k / longctx with the LM head stored as e4m3 codes and
+             power-of-two row scales (the FP8 deployment the pages report)
 
 Weights are N(0, std) with std = 1/sqrt(fan_in), fan_in being the contraction
 dimension of the matrix; the embedding table uses std 1 (a one-hot lookup reads
@@ -53,6 +55,8 @@ class Config:
     moe_inter: int = 0
     n_shared: int = 0
     stop_entropy: float = 0.05
+    lm_fp8: bool = False           # LM head stored as e4m3 codes with power-of-two row scales
+    n_layers: int = 0              # 0: one layer, unstacked arrays; L >= 1: L layers stacked [L][...]
 
     @property
     def M(self):
@@ -75,6 +79,8 @@ CONFIGS = {
                   _seeds(5, 1), inv_temp="loguniform", n_experts=128, top_k=8,
                   moe_inter=704, n_shared=1),
 }
+CONFIGS["vocab262k_fp8"] = replace(CONFIGS["vocab262k"], name="vocab262k_fp8", lm_fp8=True)
+CONFIGS["longctx_fp8"] = replace(CONFIGS["longctx"], name="longctx_fp8", lm_fp8=True)
 CONFIG_ORDER = ["tiny", "canvas256", "vocab262k", "longctx", "moe"]
 
 
@@ -98,6 +104,20 @@ def f32_to_bf16_bits(x):
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
     lsb = (u >> np.uint32(16)) & np.uint32(1)
     return ((u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+
+
+def e4m3_rows(w):
+    """Rows of a float32 matrix as e4m3 byte codes times power-of-two row
+    scales: the scale of a row is 2^ceil(log2(max|row| / 448)) (doubled if
+    rounding left it too small), the codes are torch's float8_e4m3fn cast of
+    row / scale. Returns (codes uint8, scales float32)."""
+    import torch
+    amax = np.max(np.abs(w), axis=1).astype(np.float64)
+    e = np.where(amax > 0, np.ceil(np.log2(np.maximum(amax, 1e-300) / 448.0)), 0.0)
+    e = np.where(amax * np.exp2(-e) > 448.0, e + 1, e)
+    scaled = w.astype(np.float64) * np.exp2(-e)[:, None]
+    codes = torch.from_numpy(scaled).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return codes, np.exp2(e).astype(np.float32)
 
 
 def bf16_bits_to_f32(b):
@@ -147,11 +167,25 @@ def make_workload(cfg, weight_overrides=None):
             w[name] = normal(c.weight_seed, _TID[name] if tid is None else tid, shape, std, dt)
 
     draw("embed", (c.V, c.d), 1.0)
-    draw("wq", (c.Hq * c.h, c.d), 1.0 / math.sqrt(c.d))
-    draw("wk", (c.Hk * c.h, c.d), 1.0 / math.sqrt(c.d))
-    draw("wv", (c.Hk * c.h, c.d), 1.0 / math.sqrt(c.d))
-    draw("wo", (c.d, c.Hq * c.h), 1.0 / math.sqrt(c.Hq * c.h))
-    draw("lm_head", (c.V, c.d), 1.0 / math.sqrt(c.d))
+    layer_shapes = (("wq", (c.Hq * c.h, c.d), 1.0 / math.sqrt(c.d)), ("wk", (c.Hk * c.h, c.d), 1.0 / math.sqrt(c.d)),
+                    ("wv", (c.Hk * c.h, c.d), 1.0 / math.sqrt(c.d)),
+                    ("wo", (c.d, c.Hq * c.h), 1.0 / math.sqrt(c.Hq * c.h)))
+    if c.n_layers:  # layer l > 0 draws from its own streams (tensor id + 1000 l)
+        for name, shape, std in layer_shapes:
+            if name in ov:
+                w[name] = ov.pop(name)
+                continue
+            w[name] = np.stack([normal(c.weight_seed, _TID[name] + 1000 * l, shape, std, dt)
+                                for l in range(c.n_layers)])
+    else:
+        for name, shape, std in layer_shapes:
+            draw(name, shape, std)
+    if c.lm_fp8 and "lm_head" not in ov:
+        # the same draw as the storage-dtype LM head, stored as e4m3
+        w["lm_head"], w["lm_head_scale"] = e4m3_rows(
+            normal(c.weight_seed, _TID["lm_head"], (c.V, c.d), 1.0 / math.sqrt(c.d), "f32"))
+    else:
+        draw("lm_head", (c.V, c.d), 1.0 / math.sqrt(c.d))
     if c.n_experts:
         ne = c.n_experts + c.n_shared
         draw("w_router", (c.n_experts, c.d), 1.0 / math.sqrt(c.d))
@@ -177,11 +211,14 @@ def make_workload(cfg, weight_overrides=None):
     for b in range(c.B):
         S = c.S[b]
         for lst, tid in ((pk, 10 + 2 * b), (pv, 11 + 2 * b)):
-            rng = _rng(c.weight_seed, tid)
-            x = rng.standard_normal((S, c.Hk, c.h), dtype=np.float32)
-            if scales is not None:
-                x *= scales[b][None, :, None]
-            lst.append(f32_to_bf16_bits(x) if dt == "bf16" else x)
+            per_layer = []
+            for l in range(max(1, c.n_layers)):  # [L][S][Hk][h] per request with n_layers
+                rng = _rng(c.weight_seed, tid + 1000 * l)
+                x = rng.standard_normal((S, c.Hk, c.h), dtype=np.float32)
+                if scales is not None:
+                    x *= scales[b][None, :, None]
+                per_layer.append(f32_to_bf16_bits(x) if dt == "bf16" else x)
+            lst.append(np.stack(per_layer) if c.n_layers else per_layer[0])
 
     if c.inv_temp == "loguniform":
         T = np.exp(_rng(c.weight_seed, _TID["inv_temp"]).uniform(

@@ -212,9 +212,33 @@ def moe_route(model, Hs, choice=None):
     return r, order, gates
 
 
+def dequant_rows_e4m3(codes, scales):
+    """e4m3 codes times their power-of-two row scales (exact)."""
+    return e4m3_to_f64(codes) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def fp8_matmul_rows(x, w_codes, w_scales):
+    """x W^T with W stored as e4m3 codes and row scales, x quantized per row to
+    e4m3 with its own power-of-two scale (as the FP8 LM head); both sides are
+    dequantized exactly, so the fp64 product is the exact FP8 product."""
+    qx, ex = quantize_rows_e4m3(x)
+    return dequant_rows_e4m3(qx, np.exp2(ex.astype(np.float64))) @ dequant_rows_e4m3(w_codes, w_scales).T
+
+
 def expert_ffn(model, e, x):
-    """FFN_e(x) = W_down (GELU(W_gate x) * (W_up x)); intermediate rounded to storage."""
+    """FFN_e(x) = W_down (GELU(W_gate x) * (W_up x)); intermediate rounded to storage.
+
+    With e4m3 expert weights (model["w_gate_scale"] present: w_gate, w_up and
+    w_down hold e4m3 codes with power-of-two scales per output row) each of
+    the three products is an FP8 one: the token rows are quantized per row for
+    the gate and up projections, and the intermediate (after its rounding to
+    the storage dtype) per row for the down projection."""
     dt = model["dtype"]
+    if "w_gate_scale" in model:
+        g = fp8_matmul_rows(x, model["w_gate"][e], model["w_gate_scale"][e])
+        u = fp8_matmul_rows(x, model["w_up"][e], model["w_up_scale"][e])
+        a = round_storage(gelu_exact(g) * u, dt)
+        return fp8_matmul_rows(a, model["w_down"][e], model["w_down_scale"][e])
     g = x @ widen(model["w_gate"][e], dt).T
     u = x @ widen(model["w_up"][e], dt).T
     a = round_storage(gelu_exact(g) * u, dt)

@@ -722,3 +722,37 @@ def test_second_layer_with_zero_output_projection_is_the_identity():
     # and a non-zero second layer changes them
     e3, *_ = om.forward(oracle_model(wl2), pre2, st["tok"], None)
     assert not np.allclose(e3, e1)
+
+
+def test_fp8_expert_ffn_worked_by_hand():
+    """One expert, d = 2, I = 1, e4m3 weights that are exact at scale 1:
+    gate row (1, 0), up row (0, 1), down column (1, -0.5). The token (1.5, 2)
+    is exact in e4m3 at its scale 2^-7 (192 and 256), so g = 1.5 and u = 2;
+    GELU(1.5) u = 2 * 1.5 * Phi(1.5) = 2.79957... rounds to the bf16 value
+    2.796875, whose e4m3 quantization at scale 2^-7 is 358 -> 352, i.e. 2.75;
+    the output is 2.75 * (1, -0.5) = (2.75, -1.375)."""
+    m = {"dtype": "bf16", "n_experts": 1, "top_k": 1, "moe_inter": 1, "n_shared": 0,
+         "w_gate": on.round_to_e4m3(np.array([[[1.0, 0.0]]])), "w_gate_scale": np.ones((1, 1)),
+         "w_up": on.round_to_e4m3(np.array([[[0.0, 1.0]]])), "w_up_scale": np.ones((1, 1)),
+         "w_down": on.round_to_e4m3(np.array([[[1.0], [-0.5]]])), "w_down_scale": np.ones((1, 2))}
+    y = om.expert_ffn(m, 0, np.array([[1.5, 2.0]]))
+    assert 2 * 1.5 * 0.5 * (1 + math.erf(1.5 / math.sqrt(2))) == pytest.approx(2.79957, abs=1e-5)
+    assert y.tolist() == [[2.75, -1.375]]
+    # the storage-dtype expert with the same (dequantized) weights keeps 2.796875
+    m16 = {"dtype": "bf16", "w_gate": np.array([[[1.0, 0.0]]]), "w_up": np.array([[[0.0, 1.0]]]),
+           "w_down": np.array([[[1.0], [-0.5]]])}
+    assert om.expert_ffn(m16, 0, np.array([[1.5, 2.0]])).tolist() == [[2.796875, -1.3984375]]
+
+
+def test_fp8_rows_matmul_is_the_exact_scaled_integer_sum():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((3, 96))
+    w = rng.integers(0, 126, (4, 96)).astype(np.uint8)  # non-negative finite codes
+    sw = np.exp2(rng.integers(-6, 3, 4).astype(float))
+    got = om.fp8_matmul_rows(x, w, sw)
+    qx, ex = on.quantize_rows_e4m3(x)
+    for i in range(3):
+        for j in range(4):
+            n = sum(int(round(a * 512)) * int(round(b * 512))
+                    for a, b in zip(on.e4m3_to_f64(qx[i]), on.e4m3_to_f64(w[j])))
+            assert got[i, j] == n * 2.0 ** -18 * 2.0 ** ex[i] * sw[j]

@@ -36,7 +36,8 @@ BLOCK_STEPS = 48
 REF_BUDGET_S = 150.0  # target wall time of the whole reference-arm run
 # per workload: (timed steps, warm-up steps, e2e decode blocks) when not given
 DEFAULTS = {"tiny": (4800, 96, 20), "canvas256": (4800, 96, 20), "vocab262k": (480, 48, 4),
-            "longctx": (240, 24, 2), "moe": (480, 48, 4)}
+            "longctx": (240, 24, 2), "moe": (480, 48, 4), "vocab262k_fp8": (480, 48, 4),
+            "longctx_fp8": (480, 48, 2), "moe_fp8": (480, 48, 4)}
 SUSTAINED_AFTER_S = 1.0  # a kernel timed over a region at least this long takes the sustained peak
 
 
@@ -149,7 +150,8 @@ def workload_cfg(name):
 
 def workload_label(cfg):
     moe = (f", MoE {cfg.n_experts}+{cfg.n_shared} experts top-{cfg.top_k} I{cfg.moe_inter}"
-           if cfg.n_experts else "")
+           if cfg.n_experts else "") + (", e4m3 LM head" if cfg.lm_fp8 else "") + \
+        (", e4m3 experts" if cfg.moe_fp8 else "")
     return (f"{cfg.name}: B{cfg.B} C{cfg.C} S{cfg.S[0]} d{cfg.d} Hq{cfg.Hq}/Hk{cfg.Hk} h{cfg.h} V{cfg.V} "
             f"{cfg.dtype}{moe}, {cfg.max_steps}-step blocks, adaptive stop off")
 
@@ -175,10 +177,12 @@ def flops_bytes(cfg):
     if cfg.n_experts:
         I = cfg.moe_inter
         f_moe = 2 * M * d * cfg.n_experts + M * (cfg.top_k + cfg.n_shared) * 6 * d * I
-        b_moe = (cfg.n_experts + cfg.n_shared) * 3 * d * I * es + cfg.n_experts * d * es
-    b_lm = V * d * es + M * d * es + M * 148 * 32
+        ex_es = 1 if getattr(cfg, "moe_fp8", False) else es  # e4m3 expert codes
+        b_moe = (cfg.n_experts + cfg.n_shared) * 3 * d * I * ex_es + cfg.n_experts * d * es
+    lm_es = 1 if getattr(cfg, "lm_fp8", False) else es  # e4m3 codes: one byte per weight
+    b_lm = V * d * lm_es + M * d * lm_es + V * 4 * (lm_es == 1) + M * 148 * 32
     b_attn = 2 * S * kd * es + M * (2 * qd + 2 * kd) * es
-    b_step = ((qd + 2 * kd) * d + d * qd + V * d) * es + 2 * S * kd * es + M * d * es * 6 + b_moe
+    b_step = ((qd + 2 * kd) * d + d * qd) * es + V * d * lm_es + 2 * S * kd * es + M * d * es * 6 + b_moe
     return {"flops_step": f_qkv + f_attn + f_wo + f_lm + f_moe, "bytes_step": b_step,
             "flops_lm": f_lm, "bytes_lm": b_lm, "flops_attn": f_attn, "bytes_attn": b_attn}
 
@@ -195,12 +199,17 @@ def cpu_cores_used():
 
 
 def oracle_model_of(cfg, wl):
-    """The oracle's model dictionary for a workload (MoE weights included)."""
+    """The oracle's model dictionary for a workload (MoE and e4m3 LM-head
+    weights included)."""
     m = {"dtype": cfg.dtype, "d": cfg.d, "Hq": cfg.Hq, "Hk": cfg.Hk, "h": cfg.h, "V": cfg.V}
     m.update({k: wl.weights[k] for k in ("embed", "wq", "wk", "wv", "wo", "lm_head")})
+    if cfg.lm_fp8:
+        m["lm_head_e4m3"], m["lm_head_scale"] = wl.weights["lm_head"], wl.weights["lm_head_scale"]
     if cfg.n_experts:
         m.update(n_experts=cfg.n_experts, top_k=cfg.top_k, moe_inter=cfg.moe_inter, n_shared=cfg.n_shared)
         m.update({k: wl.weights[k] for k in ("w_router", "w_gate", "w_up", "w_down")})
+        if cfg.moe_fp8:
+            m.update({k: wl.weights[k] for k in ("w_gate_scale", "w_up_scale", "w_down_scale")})
     return m
 
 
@@ -210,7 +219,8 @@ def oracle_step_timer(cfg, wl):
     the block when it is done. Weights and prefix K/V are widened to fp64
     first (outside the timed calls)."""
     from oracle import model as om
-    m = om.prewiden(oracle_model_of(cfg, wl))
+    m = oracle_model_of(cfg, wl)
+    m = om.prewiden(m, ("wq", "wk", "wv", "wo") if cfg.lm_fp8 else ("wq", "wk", "wv", "wo", "lm_head"))
     prefix = [(om.widen(k, cfg.dtype), om.widen(v, cfg.dtype)) for k, v in zip(wl.prefix_k, wl.prefix_v)]
     sched = {"max_steps": cfg.max_steps, "stop_entropy": cfg.stop_entropy, "adaptive_stop": False}
 
@@ -314,13 +324,20 @@ def bench_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------- b200 arm
-def kernel_roofline(name, kernel, flops, bytes_, avg_ms, peaks, peak_kind, traffic):
-    peak = peaks["bf16_tflops_sustained"] if peak_kind == "sustained" else peaks["bf16_tflops"]
+FP8_OVER_BF16 = 2.0  # nominal dense ratio 4.5 / 2.25 PFLOP/s
+
+
+def kernel_roofline(name, kernel, flops, bytes_, avg_ms, peaks, peak_kind, traffic, fp8=False):
+    """A contraction's roofline against the peak of its own operand type: the
+    measured bf16 peak, times the nominal FP8/bf16 ratio for e4m3 operands."""
+    mult = FP8_OVER_BF16 if fp8 else 1.0
+    peak = mult * (peaks["bf16_tflops_sustained"] if peak_kind == "sustained" else peaks["bf16_tflops"])
     tflops = flops / (avg_ms / 1e3) / 1e12
-    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    t_roof = max(flops / (mult * peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
     return {"bound": "tensor", "kernel": kernel, "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
             "frac": tflops / peak, "traffic": traffic,
-            "peak_source": f"{peaks['source']} {peak_kind} bf16 ("
+            "peak_source": f"{peaks['source']} {peak_kind} bf16"
+                           + (" x 2 (nominal e4m3/bf16 dense ratio)" if fp8 else "") + " ("
                            + ("kernel timed inside a step loop of a second or more"
                               if peak_kind == "sustained" else "kernel timed inside a step loop shorter than 1 s")
                            + ")",
@@ -425,8 +442,10 @@ def bench_b200(args, rank, world, local_rank):
         cv.set_timing_events([], [], kernel=k)
     steps_per_s = job_rate(args.steps, world, elapsed_ms)
     peak_kind = "sustained" if region2_s >= SUSTAINED_AFTER_S else "burst"
-    lm = kernel_roofline("lmhead", "lmhead_tc_kernel (LM head + entropy/argmax)", fb["flops_lm"], fb["bytes_lm"],
-                         float(np.mean(dur["lmhead"])), peaks, peak_kind, traffic_of("lmhead_tc_kernel", cfg.name))
+    lm = kernel_roofline("lmhead", "lmhead_tc_kernel<" + ("e4m3" if cfg.lm_fp8 else "bf16")
+                         + "> (LM head + entropy/argmax)", fb["flops_lm"], fb["bytes_lm"],
+                         float(np.mean(dur["lmhead"])), peaks, peak_kind, traffic_of("lmhead_tc_kernel", cfg.name),
+                         fp8=cfg.lm_fp8)
     at = kernel_roofline("attention", "attn_tc_kernel (+ attn_merge_kernel when split)", fb["flops_attn"],
                          fb["bytes_attn"], float(np.mean(dur["attention"])), peaks, peak_kind,
                          traffic_of("attn_tc_kernel", cfg.name))
@@ -488,7 +507,8 @@ def bench_b200(args, rank, world, local_rank):
             "roofline": lm,
             "rooflines": {"lmhead": lm, "attention": at},
             "step_roofline": {"flops": fb["flops_step"], "bytes": fb["bytes_step"],
-                              "ms": max(fb["flops_step"] / (peaks["bf16_tflops"] * 1e12),
+                              "ms": max((fb["flops_step"] - fb["flops_lm"] * (1 - 1 / FP8_OVER_BF16) * cfg.lm_fp8)
+                                        / (peaks["bf16_tflops"] * 1e12),
                                         fb["bytes_step"] / (peaks["hbm_gbs"] * 1e9)) * 1e3},
             "kernel_timing_region_s": region2_s,
             "cpu_baseline": cpu,

@@ -39,7 +39,7 @@
  *     error word that the next synchronous call reports as
  *     DG_ERR_DEVICE_CHECK / DG_ERR_TIMEOUT; kernels never trap.
  *   - A context must not be used from two host threads at once.
- *   - Shapes supported: canvas_len 1..256; storage dtype f32 (CUDA-core
+ *   - Shapes supported: canvas_len 1..1024; storage dtype f32 (CUDA-core
  *     kernels, head_dim 32..128 multiple of 32) or bf16 (tensor-core kernels,
  *     head_dim 128, d_model a multiple of 64, vocab a multiple of 256,
  *     n_q_heads a multiple of n_kv_heads).
@@ -93,7 +93,37 @@ typedef struct dg_model_desc {
   const void *w_gate;   /* [n_experts+n_shared][moe_inter][d_model] */
   const void *w_up;     /* [n_experts+n_shared][moe_inter][d_model] */
   const void *w_down;   /* [n_experts+n_shared][d_model][moe_inter] */
+  /* Storage of lm_head (the FP8 deployment of [P3] 性能数据 and [P4]
+   * 引入扩散机制): DG_LM_STORAGE (0) = the storage dtype; DG_LM_E4M3 (1) =
+   * e4m3 byte codes [vocab][d_model] with lm_head_scale[v] (device, [vocab]
+   * f32, a power of two) the scale of row v. With DG_LM_E4M3 each row r of
+   * the residual stream is quantized to e4m3 with the smallest power-of-two
+   * scale s_r that fits its largest magnitude (round to nearest, ties to
+   * even) and the logits are s_r lm_head_scale[v] (q_r . q_v), f32
+   * accumulate. Needs the bf16 dtype and d_model % 128 == 0. */
+  int32_t lm_head_format;
+  const float *lm_head_scale;
+  /* Attention layers ([P3] 局限 2 raises deeper and longer variants): 0 or 1
+   * = the single layer above; L > 1 = L layers in sequence, each the single
+   * layer (Q/K/V of its input, bidirectional attention over its own prompt
+   * K/V and the canvas, Wo + residual) fed the previous layer's output, the
+   * LM head reading the last. wq, wk, wv, wo then hold the L layers stacked
+   * layer-major ([L][out][in]) and each request's prompt K/V cache is
+   * [L][S_b][n_kv_heads][head_dim]. L <= 64; not with the MoE block. */
+  int32_t n_layers;
+  /* Storage of the expert weights: DG_LM_STORAGE (0) = the storage dtype;
+   * DG_LM_E4M3 (1) = w_gate, w_up, w_down hold e4m3 byte codes and
+   * w_gate_scale / w_up_scale ([n_experts+n_shared][moe_inter] f32) and
+   * w_down_scale ([n_experts+n_shared][d_model] f32) their per-row scales
+   * (powers of two). The token rows are then quantized per row (as for the
+   * e4m3 LM head) for the gate and up projections, and the GeGLU product,
+   * after its rounding to the storage dtype, per row for the down
+   * projection; f32 accumulate. Needs d_model % 128 == 0. */
+  int32_t expert_format;
+  const float *w_gate_scale, *w_up_scale, *w_down_scale;
 } dg_model_desc;
+#define DG_LM_STORAGE 0
+#define DG_LM_E4M3 1
 
 /* Freeze schedule and stop rule ([P1] 整片并行去噪, 自适应停步机制).
  * At step t of a canvas with U unfrozen positions, k = ceil(U / (max_steps - t))
@@ -120,6 +150,8 @@ typedef struct dg_step_out {
   void *q;              /* [B*C][n_q_heads*head_dim] queries (dtype)           */
   void *k_canvas;       /* [B*C][n_kv_heads*head_dim] canvas keys (dtype)      */
   void *v_canvas;       /* [B*C][n_kv_heads*head_dim] canvas values (dtype)    */
+  void *layer_out;      /* [L][B*C][d_model] residual stream after each layer;
+                           q, k_canvas, v_canvas, attn_out are the last layer's */
 } dg_step_out;
 
 /* Host-side copy of the decode state (all host arrays). */
@@ -136,10 +168,12 @@ typedef struct dg_ctx dg_ctx;
 /* Create a decode context and draw the initial canvases.
  *   model       weights (see dg_model_desc); copied by value.
  *   batch       B >= 1 independent canvases (requests).
- *   canvas_len  C, 1..256 positions per canvas.
+ *   canvas_len  C, 1..1024 positions per canvas (the pages use 256; longer
+ *               canvases are an open question there: [P3] 局限).
  *   prefix_len  host [B]: cached prompt length S_b >= 0 of each request.
  *   prefix_k/v  host arrays of B device pointers, each [S_b][n_kv_heads][head_dim]
- *               in the storage dtype (NULL allowed when S_b = 0).
+ *               in the storage dtype ([L][S_b][...] with n_layers = L > 1; NULL
+ *               allowed when S_b = 0).
  *   inv_temp    device [B*C] f32 per-position inverse temperature applied to the
  *               logits before the entropy, or NULL for 1.
  *   seeds       host [B] Philox seeds; canvas b position p starts at
@@ -223,10 +257,14 @@ dg_status dg_canvas_set_state(dg_ctx *ctx, const dg_state *host_in);
  * stops[i % n] just after the kernel named by `kernel`: DG_KERNEL_LMHEAD (the
  * LM head with its entropy/argmax epilogue) or DG_KERNEL_ATTENTION (the
  * attention kernel, with its split-KV merge when it has one). n = 0 turns it
- * off for that kernel; the two kernels' settings are independent.
- * Synchronous (drops the captured step graphs). Not used by dg_decode_block. */
+ * off for that kernel; the settings are independent. DG_KERNEL_DECODE takes
+ * one pair (n <= 1), recorded by dg_decode_block's graph just before its loop
+ * starts and just after it ends (the device time of the loop alone); the
+ * kernel pairs are not recorded inside that loop.
+ * Synchronous (drops the captured graphs). */
 #define DG_KERNEL_LMHEAD 0
 #define DG_KERNEL_ATTENTION 1
+#define DG_KERNEL_DECODE 2
 dg_status dg_canvas_set_kernel_timing(dg_ctx *ctx, int32_t kernel, int32_t n, void *const *starts,
                                       void *const *stops);
 /* dg_canvas_set_kernel_timing(ctx, DG_KERNEL_LMHEAD, n, starts, stops). */

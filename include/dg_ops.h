@@ -35,6 +35,23 @@ extern "C" {
 dg_status dg_lmhead_entropy(int32_t dtype, const void *hs, const void *lm_head, const float *inv_temp,
                             int32_t M, int32_t d, int32_t V, float *ent, int32_t *argmax, void *stream);
 
+/* The LM head with e4m3 weights (the FP8 deployment of [P3] 性能数据):
+ * each row of hs (bf16 [M][d]) is quantized to e4m3 with the smallest
+ * power-of-two scale s_r that fits its largest magnitude (round to nearest,
+ * ties to even), and
+ *   x[r][v] = s_r lm_scale[v] (q_r . q_v)   (f32 accumulate)
+ * with lm_head e4m3 byte codes [V][d] and lm_scale [V] f32 row scales
+ * (powers of two); then ent and argmax as in dg_lmhead_entropy.
+ * Needs d % 128 == 0 and V % 256 == 0. */
+dg_status dg_lmhead_entropy_e4m3(const void *hs, const void *lm_head, const float *lm_scale, const float *inv_temp,
+                                 int32_t M, int32_t d, int32_t V, float *ent, int32_t *argmax, void *stream);
+
+/* The quantization step of dg_lmhead_entropy_e4m3 alone: each row r of x
+ * (bf16 [M][d]) becomes e4m3 codes [M][d] (bytes) and scales[r] (f32, the
+ * smallest power of two s with 448 s >= max |x[r]|), codes = x[r] / s
+ * rounded to the nearest e4m3 value, ties to even. d % 8 == 0. */
+dg_status dg_quantize_rows_e4m3(const void *x, uint8_t *codes, float *scales, int32_t M, int32_t d, void *stream);
+
 /* Allocation-free variant of dg_lmhead_entropy. The pages have no counterpart
  * to this call: it exists for callers of this library that cannot allocate
  * device memory where they run the LM head -- an application whose device

@@ -19,6 +19,9 @@ def oracle_model(wl):
                  n_shared=c.n_shared)
         for k in ("w_router", "w_gate", "w_up", "w_down"):
             m[k] = wl.weights[k]
+        if c.moe_fp8:  # e4m3 expert codes with row scales
+            for k in ("w_gate_scale", "w_up_scale", "w_down_scale"):
+                m[k] = wl.weights[k]
     return m
 
 

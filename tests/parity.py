@@ -126,9 +126,24 @@ def route_choices(r_row, k):
 
 def check_tensor_stages(cfg, omodel, oprefix, tok, gpu, rep):
     """Q/K/V, attention, Wo + residual and MoE, each against the oracle fed
-    the GPU's own input to that stage."""
+    the GPU's own input to that stage. With a stack of L layers, layer l < L-1
+    is compared as a whole (its output against the oracle's layer l fed the
+    GPU's input to it) and the last layer stage by stage."""
     B, C = cfg.B, cfg.C
+    L = om.n_layers(omodel)
     X = om.embed(omodel, tok)
+    lo = gpu.get("layer_out")
+    for l in range(L - 1):
+        ref = om.attention_layer(omodel, oprefix, X, B, C, l)[4]
+        n, mx = close(lo[l], ref)
+        rep.dev(f"layer{l}_out", mx)
+        if n:
+            rep.fail(f"layer {l} output: {n} elements out of tolerance (max abs diff {mx:.3g})")
+        X = lo[l].astype(np.float64)
+    if lo is not None and not np.array_equal(lo[L - 1], gpu["hidden_attn"]):
+        rep.fail("the last layer's output differs from hidden_attn")
+    last, oprefix = om.layer(omodel, L - 1), om.layer_prefix(omodel, oprefix, L - 1)
+    omodel = last
     Qo, Kco, Vco = om.project_qkv(omodel, X)
     for name, g, o in (("q", gpu["q"], Qo), ("k_canvas", gpu["k_canvas"], Kco), ("v_canvas", gpu["v_canvas"], Vco)):
         n, mx = close(g, o.reshape(g.shape))

@@ -119,7 +119,7 @@ def test_init_rejects_moe_beyond_one_routing_block(lib):
     assert not ctx.value
 
 
-@pytest.mark.parametrize("batch,canvas", [(0, 16), (1, 0), (1, 257)])
+@pytest.mark.parametrize("batch,canvas", [(0, 16), (1, 0), (1, 1025)])
 def test_init_rejects_bad_sizes(lib, batch, canvas):
     m = _model()
     ctx = C.c_void_p()

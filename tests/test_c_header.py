@@ -13,10 +13,11 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 STRUCTS = {
     "dg_model_desc": ["d_model", "vocab", "dtype", "embed", "lm_head", "n_experts", "n_shared", "w_router",
-                      "w_down"],
+                      "w_down", "lm_head_format", "lm_head_scale", "n_layers", "expert_format",
+                      "w_down_scale"],
     "dg_schedule": ["max_steps", "stop_entropy", "adaptive_stop", "kind"],
     "dg_step_out": ["ent", "argmax", "freeze_mask", "attn_out", "hidden", "hidden_attn", "q", "k_canvas",
-                    "v_canvas"],
+                    "v_canvas", "layer_out"],
     "dg_state": ["tokens", "frozen", "step", "seed", "done"],
 }
 
@@ -28,7 +29,8 @@ def _program():
              "  /* reference the entry points so that the link resolves them */",
              "  fn volatile f[] = {(fn)dg_canvas_init, (fn)dg_denoise_step, (fn)dg_decode_block,",
              "                     (fn)dg_canvas_reset_fixed, (fn)dg_canvas_block_kv, (fn)dg_canvas_set_prefix,",
-             "                     (fn)dg_lmhead_entropy, (fn)dg_lmhead_entropy_noalloc, (fn)dg_attention,",
+             "                     (fn)dg_lmhead_entropy, (fn)dg_lmhead_entropy_e4m3,",
+             "                     (fn)dg_quantize_rows_e4m3, (fn)dg_lmhead_entropy_noalloc, (fn)dg_attention,",
              "                     (fn)dg_linear, (fn)dg_ops_check, (fn)dg_selftest_wait_timeout};",
              "  (void)f;"]
     for s, fields in STRUCTS.items():

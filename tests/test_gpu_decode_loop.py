@@ -6,7 +6,8 @@ launch) and runs no step after the stop ("DiffusionGemma解析：扩散模型如
 
 On the canvas256 workload: a stop threshold above every entropy stops each
 block after its first step (k = 1); without the adaptive stop the block runs
-its whole schedule (k = 6 and k = 48). The block's device time must be at most
+its whole schedule (k = 6 and k = 48). The loop's device time (events the
+decode graph records just before and after its loop) must be at most
 (k + 0.2) times one step's time, measured from back-to-back graph steps."""
 import numpy as np
 import pytest
@@ -37,16 +38,18 @@ def test_decode_block_runs_exactly_the_steps_it_needs():
         e1.record(stream)
         torch.cuda.synchronize()
         t_step = e0.elapsed_time(e1) / n
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)  # torch creates the CUDA events on their first record
+        d1.record(stream)
+        cv.set_timing_events([d0], [d1], kernel="decode")
         cases = [(schedule(48, 100.0, True), 1), (schedule(6, 0.05, False), 6), (schedule(48, 0.05, False), 48)]
         for sched, k in cases:
             cv.reset()
             cv.decode(sched)  # builds the decode graph for this schedule
             cv.reset()
-            e0.record(stream)
             toks, steps = cv.decode(sched)
-            e1.record(stream)
             torch.cuda.synchronize()
-            t = e0.elapsed_time(e1)
+            t = d0.elapsed_time(d1)
             st = cv.get_state()
             print(f"k={k}: decode {t:.3f} ms, one step {t_step:.4f} ms, ratio {t / t_step:.2f}")
             assert steps == [k] and np.all(st["step"] == k) and np.all(st["done"]) and np.all(st["frozen"])

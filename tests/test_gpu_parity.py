@@ -66,6 +66,51 @@ def test_bf16_canvas256_first_steps_lockstep():
     _run(fx.CONFIGS["canvas256"], n_steps=3, free_running=False)
 
 
+@pytest.mark.parametrize("dtype,B,C", [("bf16", 2, 512), ("bf16", 1, 1000), ("f32", 1, 1024)])
+def test_long_canvas_full_decode(dtype, B, C):
+    """Canvases longer than the pages' 256 positions (512 and 1024 are the
+    lengths raised as an open question: "DiffusionGemma深度拆解", 局限 2): the
+    selection sorts up to 1024 keys per canvas; full free-running decode,
+    ragged (1000 = 7 tiles of 128 + 104) and exact tile multiples."""
+    if dtype == "bf16":
+        cfg = fx.Config(f"long_canvas_{C}", B=B, C=C, S=tuple([200, 0][:B]), d=128, Hq=2, Hk=1, h=128, V=2048,
+                        dtype="bf16", max_steps=16, weight_seed=51, canvas_seeds=tuple(8 + b for b in range(B)))
+    else:
+        cfg = fx.Config(f"long_canvas_f32_{C}", B=B, C=C, S=(40,), d=64, Hq=2, Hk=1, h=32, V=512, dtype="f32",
+                        max_steps=12, weight_seed=52, canvas_seeds=(3,))
+    _, steps = _run(cfg)
+    assert 1 <= steps <= cfg.max_steps
+
+
+@pytest.mark.parametrize("dtype,L", [("bf16", 3), ("f32", 2)])
+def test_layer_stack_full_decode(dtype, L):
+    """A stack of attention layers, each over its own prompt K/V
+    ("DiffusionGemma深度拆解", 局限 2 and 架构解剖 1): every inner layer's output and
+    the last layer's stages against the oracle fed the GPU's inputs, full
+    free-running decode."""
+    if dtype == "bf16":
+        cfg = fx.Config("layers_bf16", B=2, C=150, S=(100, 40), d=128, Hq=2, Hk=1, h=128, V=2048, dtype="bf16",
+                        max_steps=10, weight_seed=81, canvas_seeds=(4, 5), n_layers=L)
+    else:
+        cfg = fx.Config("layers_f32", B=2, C=24, S=(10, 33), d=64, Hq=2, Hk=1, h=32, V=300, dtype="f32",
+                        max_steps=7, weight_seed=82, canvas_seeds=(1, 2), n_layers=L)
+    _, steps = _run(cfg)
+    assert 1 <= steps <= cfg.max_steps
+
+
+def test_block_kv_needs_the_single_layer_model():
+    from token_canvas_denoising_b200 import _lib as L
+    cfg = fx.Config("layers_kv", B=1, C=16, S=(8,), d=64, Hq=2, Hk=1, h=32, V=64, dtype="f32", max_steps=4,
+                    weight_seed=83, canvas_seeds=(1,), n_layers=2)
+    cv, keep = _canvas(fx.make_workload(cfg))
+    try:
+        with pytest.raises(L.DgError) as e:
+            cv.block_kv()
+        assert e.value.status == L.DG_ERR_UNSUPPORTED
+    finally:
+        cv.close()
+
+
 def test_bf16_moe_small_full_decode():
     """MoE FFN path (router, top-k routing, GeGLU experts, shared expert,
     combine) on a small model, full decode."""

@@ -48,8 +48,11 @@ def test_route_choices_enumerate_the_near_ties_only():
 
 
 # ---------------------------------------------------------------- check_step on oracle-made outputs
-def _small_case(moe=False, adaptive=False):
-    if moe:
+def _small_case(moe=False, adaptive=False, layers=0):
+    if layers:
+        cfg = fx.Config("h_layers", B=2, C=12, S=(7, 0), d=32, Hq=2, Hk=1, h=16, V=64, dtype="f32", max_steps=5,
+                        weight_seed=43, canvas_seeds=(3, 4), n_layers=layers)
+    elif moe:
         cfg = fx.Config("h_moe", B=2, C=12, S=(7, 0), d=32, Hq=2, Hk=1, h=16, V=64, dtype="f32", max_steps=5,
                         weight_seed=41, canvas_seeds=(3, 4), n_experts=6, top_k=2, moe_inter=16, n_shared=1)
     else:
@@ -72,13 +75,14 @@ def _fake_gpu_step(cfg, m, pre, sched, st):
     gpu = {"ent": rec["ent"].reshape(-1).astype(np.float32), "argmax": rec["am"].reshape(-1).astype(np.int32),
            "freeze_mask": fm.reshape(-1).astype(np.uint8), "attn_out": ex["O"],
            "hidden": ex["Hs"], "hidden_attn": ex["Hs_attn"], "q": ex["Q"].reshape(B * C, -1),
-           "k_canvas": ex["Kc"].reshape(B * C, -1), "v_canvas": ex["Vc"].reshape(B * C, -1)}
+           "k_canvas": ex["Kc"].reshape(B * C, -1), "v_canvas": ex["Vc"].reshape(B * C, -1),
+           "layer_out": np.stack(ex["layers"])}
     return gpu, pa.oracle_state_to_abi(new), new
 
 
-@pytest.mark.parametrize("moe", [False, True])
-def test_check_step_accepts_the_oracles_own_steps(moe):
-    cfg, wl, m, pre, sched = _small_case(moe)
+@pytest.mark.parametrize("moe,layers", [(False, 0), (True, 0), (False, 3)])
+def test_check_step_accepts_the_oracles_own_steps(moe, layers):
+    cfg, wl, m, pre, sched = _small_case(moe, layers=layers)
     st = om.init_state(wl.seeds, cfg.C, cfg.V)
     rep = pa.StepReport()
     while not st["done"].all():
@@ -229,3 +233,15 @@ def test_valid_choice_at_a_freeze_tie_is_followed_not_reported():
     assert not rep.errors, rep.errors
     assert rep.div_freeze == 1 and rep.diverged_steps == 1 and rep.amb_cut >= 2
     assert np.array_equal(nxt["tok"], tok) and np.array_equal(nxt["frozen"], frozen)
+
+
+def test_planted_layer_error_is_reported():
+    """A wrong output of an inner layer of a stack is reported for that layer."""
+    cfg, wl, m, pre, sched = _small_case(layers=3)
+    st = om.init_state(wl.seeds, cfg.C, cfg.V)
+    gpu, gst, _ = _fake_gpu_step(cfg, m, pre, sched, st)
+    gpu["layer_out"] = gpu["layer_out"].copy()
+    gpu["layer_out"][1, 4, 2] += 0.5
+    rep = pa.StepReport()
+    pa.check_step(cfg, m, pre, sched, None, st, gpu, gst, rep)
+    assert any("layer 1 output" in e for e in rep.errors)

@@ -12,8 +12,9 @@ LIB_PATH = os.path.join(_HERE, "libdgcanvas.so")
 DG_OK, DG_ERR_INVALID_ARG, DG_ERR_UNSUPPORTED, DG_ERR_OOM, DG_ERR_CUDA, DG_ERR_TIMEOUT, \
     DG_ERR_DEVICE_CHECK = range(7)
 DG_F32, DG_BF16 = 0, 1
+DG_LM_STORAGE, DG_LM_E4M3 = 0, 1
 DG_SCHED_CEIL = 0
-DG_KERNEL_LMHEAD, DG_KERNEL_ATTENTION = 0, 1
+DG_KERNEL_LMHEAD, DG_KERNEL_ATTENTION, DG_KERNEL_DECODE = 0, 1, 2
 
 
 class dg_model_desc(C.Structure):
@@ -24,7 +25,10 @@ class dg_model_desc(C.Structure):
                 ("n_experts", C.c_int32), ("top_k", C.c_int32), ("moe_inter", C.c_int32),
                 ("n_shared", C.c_int32),
                 ("w_router", C.c_void_p), ("w_gate", C.c_void_p), ("w_up", C.c_void_p),
-                ("w_down", C.c_void_p)]
+                ("w_down", C.c_void_p),
+                ("lm_head_format", C.c_int32), ("lm_head_scale", C.c_void_p), ("n_layers", C.c_int32),
+                ("expert_format", C.c_int32), ("w_gate_scale", C.c_void_p), ("w_up_scale", C.c_void_p),
+                ("w_down_scale", C.c_void_p)]
 
 
 class dg_schedule(C.Structure):
@@ -35,7 +39,7 @@ class dg_schedule(C.Structure):
 class dg_step_out(C.Structure):
     _fields_ = [("ent", C.c_void_p), ("argmax", C.c_void_p), ("freeze_mask", C.c_void_p),
                 ("attn_out", C.c_void_p), ("hidden", C.c_void_p), ("hidden_attn", C.c_void_p),
-                ("q", C.c_void_p), ("k_canvas", C.c_void_p), ("v_canvas", C.c_void_p)]
+                ("q", C.c_void_p), ("k_canvas", C.c_void_p), ("v_canvas", C.c_void_p), ("layer_out", C.c_void_p)]
 
 
 class dg_state(C.Structure):
@@ -68,6 +72,9 @@ SIGNATURES = {
     # include/dg_ops.h
     "dg_lmhead_entropy": (C.c_int, [C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
                                     C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_lmhead_entropy_e4m3": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32,
+                                         C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "dg_quantize_rows_e4m3": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p]),
     "dg_lmhead_entropy_noalloc": (C.c_int, [C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32,
                                             C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_lmhead_entropy_noalloc_max_records": (C.c_size_t, []),

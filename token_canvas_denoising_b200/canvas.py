@@ -20,7 +20,7 @@ def _ptr(t):
 def to_device(arr, dtype, device):
     """numpy storage array (uint16 bf16 bits or float32) -> contiguous torch tensor."""
     t = torch.from_numpy(np.ascontiguousarray(arr))
-    if dtype == "bf16":
+    if arr.dtype == np.uint16:  # bf16 bit patterns (uint8 e4m3 codes stay bytes)
         t = t.view(torch.bfloat16)
     return t.to(device, non_blocking=False).contiguous()
 
@@ -39,7 +39,7 @@ class DenoiseCanvas:
 
     def __init__(self, weights, *, d_model, n_q_heads, n_kv_heads, head_dim, vocab, dtype,
                  canvas_len, prefix_k, prefix_v, seeds, inv_temp=None, n_experts=0, top_k=0,
-                 moe_inter=0, n_shared=0, stream=None):
+                 moe_inter=0, n_shared=0, n_layers=0, stream=None):
         self._lib = L.load()
         self.B = len(seeds)
         self.C = int(canvas_len)
@@ -52,11 +52,20 @@ class DenoiseCanvas:
         for k in ("embed", "wq", "wk", "wv", "wo", "lm_head"):
             setattr(m, k, weights[k].data_ptr())
         m.n_experts, m.top_k, m.moe_inter, m.n_shared = n_experts, top_k, moe_inter, n_shared
+        m.n_layers = n_layers
+        self.L = max(1, n_layers)
+        if "lm_head_scale" in weights:  # e4m3 LM head
+            m.lm_head_format = L.DG_LM_E4M3
+            m.lm_head_scale = weights["lm_head_scale"].data_ptr()
         if n_experts:
             for k in ("w_router", "w_gate", "w_up", "w_down"):
                 setattr(m, k, weights[k].data_ptr())
+            if "w_gate_scale" in weights:  # e4m3 experts
+                m.expert_format = L.DG_LM_E4M3
+                for k in ("w_gate_scale", "w_up_scale", "w_down_scale"):
+                    setattr(m, k, weights[k].data_ptr())
         self._model = m
-        plen = (C.c_int32 * self.B)(*[int(t.shape[0]) if t is not None else 0 for t in prefix_k])
+        plen = (C.c_int32 * self.B)(*[self._plen(t) for t in prefix_k])
         pk = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_k])
         pv = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_v])
         sd = (C.c_uint64 * self.B)(*[int(s) for s in seeds])
@@ -67,6 +76,12 @@ class DenoiseCanvas:
                                       C.cast(sd, C.c_void_p), C.c_void_p(self.stream.cuda_stream))
         L.check(st, "dg_canvas_init")
         self._ctx = ctx
+
+    def _plen(self, t):
+        """Prompt length of a cache tensor ([S][Hk][h], or [L][S][Hk][h] with L layers)."""
+        if t is None:
+            return 0
+        return int(t.shape[1]) if self._model.n_layers > 0 and t.dim() == 4 else int(t.shape[0])
 
     # ------------------------------------------------------------------
     def step(self, sched, debug=False):
@@ -88,9 +103,10 @@ class DenoiseCanvas:
                 "q": torch.empty(self.M, qd, dtype=sdt, device=dev),
                 "k_canvas": torch.empty(self.M, kd, dtype=sdt, device=dev),
                 "v_canvas": torch.empty(self.M, kd, dtype=sdt, device=dev),
+                "layer_out": torch.empty(self.L, self.M, self._model.d_model, dtype=sdt, device=dev),
             }
             dbg = L.dg_step_out(*[_ptr(out[k]) for k in ("ent", "argmax", "freeze_mask", "attn_out", "hidden",
-                                                          "hidden_attn", "q", "k_canvas", "v_canvas")])
+                                                          "hidden_attn", "q", "k_canvas", "v_canvas", "layer_out")])
         st = self._lib.dg_denoise_step(self._ctx, C.byref(sched), C.byref(dbg) if dbg is not None else None)
         L.check(st, "dg_denoise_step")
         return out
@@ -158,7 +174,7 @@ class DenoiseCanvas:
     def set_prefix(self, prefix_k, prefix_v):
         """Attend to new prompt caches from the next step on: lists of B device
         tensors [S_b, Hk, h] (kept alive by this object)."""
-        plen = (C.c_int32 * self.B)(*[int(t.shape[0]) if t is not None else 0 for t in prefix_k])
+        plen = (C.c_int32 * self.B)(*[self._plen(t) for t in prefix_k])
         pk = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_k])
         pv = (C.c_void_p * self.B)(*[t.data_ptr() if t is not None and t.numel() else None for t in prefix_v])
         st = self._lib.dg_canvas_set_prefix(self._ctx, C.cast(plen, C.c_void_p), C.cast(pk, C.c_void_p),
@@ -168,9 +184,10 @@ class DenoiseCanvas:
 
     def set_timing_events(self, starts, stops, kernel="lmhead"):
         """Record torch.cuda.Event pairs around one kernel of graph steps
-        (pair i on step i mod n): kernel "lmhead" or "attention". Pass empty
+        (pair i on step i mod n): kernel "lmhead" or "attention"; or one pair
+        around the device-side loop of decode(): kernel "decode". Pass empty
         lists to turn off."""
-        k = {"lmhead": L.DG_KERNEL_LMHEAD, "attention": L.DG_KERNEL_ATTENTION}[kernel]
+        k = {"lmhead": L.DG_KERNEL_LMHEAD, "attention": L.DG_KERNEL_ATTENTION, "decode": L.DG_KERNEL_DECODE}[kernel]
         n = len(starts)
         a = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in starts])
         b = (C.c_void_p * max(n, 1))(*[e.cuda_event for e in stops])
@@ -208,5 +225,5 @@ def from_workload(wl, device=None, stream=None):
     cv = DenoiseCanvas(w, d_model=c.d, n_q_heads=c.Hq, n_kv_heads=c.Hk, head_dim=c.h, vocab=c.V,
                        dtype=c.dtype, canvas_len=c.C, prefix_k=pk, prefix_v=pv, seeds=list(wl.seeds),
                        inv_temp=invT, n_experts=c.n_experts, top_k=c.top_k, moe_inter=c.moe_inter,
-                       n_shared=c.n_shared, stream=stream)
+                       n_shared=c.n_shared, n_layers=c.n_layers, stream=stream)
     return cv, {"weights": w, "prefix_k": pk, "prefix_v": pv, "inv_temp": invT}

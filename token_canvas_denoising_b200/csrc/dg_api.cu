@@ -72,29 +72,40 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
   c->cs.counters = w.take<uint32_t>(c->B + 1);
   c->cs.loop_iter = w.take<int32_t>(1);
   c->err = w.take<int32_t>(1);
-  c->d_prefix = w.take<dg::PrefixDesc>(c->B);
-  c->X = w.take<char>(M * d * c->es);
+  c->d_prefix = w.take<dg::PrefixDesc>((size_t)c->L * c->B);  // [L][B]
+  c->xres.assign(c->L + 1, nullptr);
+  for (int l = 0; l <= c->L; ++l) c->xres[l] = w.take<char>(M * d * c->es);
+  c->X = c->xres[0];
   c->Q = w.take<char>(M * qd * c->es);
   c->Kc = w.take<char>(M * kd * c->es);
   c->Vc = w.take<char>(M * kd * c->es);
   c->O = w.take<char>(M * qd * c->es);
-  c->Hs = w.take<char>(M * d * c->es);
+  c->Hs = c->xres[c->L];
   c->Hs2 = c->m.n_experts ? w.take<char>(M * d * c->es) : nullptr;
   c->lm.rec = w.take<dg::LmRec>(M * (size_t)c->lm.P);
+  if (c->m.lm_head_format == DG_LM_E4M3) {
+    c->hs8 = w.take<uint8_t>(M * d);
+    c->hs8_scale = w.take<float>(M);
+  }
   c->ent = w.take<float>(M);
   c->am = w.take<int32_t>(M);
   if (c->m.n_experts) {
-    dg::MoeShape ms{c->M, c->m.d_model, c->m.n_experts, c->m.top_k, c->m.n_shared, c->m.moe_inter};
+    dg::MoeShape ms{c->M, c->m.d_model, c->m.n_experts, c->m.top_k, c->m.n_shared, c->m.moe_inter,
+                    c->m.expert_format == DG_LM_E4M3};
     c->moe_ws = w.take<char>(dg::moe_workspace_bytes(ms));
   }
-  if (c->m.dtype == DG_BF16) {
-    c->g_qkv.part = w.take<float>(dg::gemm_tc_partial_floats(c->g_qkv));
-    c->g_wo.part = w.take<float>(dg::gemm_tc_partial_floats(c->g_wo));
+  if (c->m.dtype == DG_BF16) {  // split-K partials, shared by the layers (same shapes)
+    float* pq = w.take<float>(dg::gemm_tc_partial_floats(c->g_qkv[0]));
+    float* po = w.take<float>(dg::gemm_tc_partial_floats(c->g_wo[0]));
+    for (int l = 0; l < c->L; ++l) {
+      c->g_qkv[l].part = pq;
+      c->g_wo[l].part = po;
+    }
   }
   if (c->m.dtype == DG_BF16 && c->attn_splits > 1) {
     const size_t rows = M * (size_t)c->m.n_q_heads;
-    c->attn.part_o = w.take<float>((size_t)c->attn_splits * rows * 128);
-    c->attn.part_ml = w.take<float>((size_t)c->attn_splits * rows * 2);
+    c->attn_part_o = w.take<float>((size_t)c->attn_splits * rows * 128);
+    c->attn_part_ml = w.take<float>((size_t)c->attn_splits * rows * 2);
   }
   *total = w.off + 256;
 }
@@ -117,6 +128,17 @@ dg_status validate_model(const dg_model_desc* m) {
     DG_UNSUP(m->d_model % 64 == 0, "bf16 d_model must be a multiple of 64");
     DG_UNSUP(m->vocab % 256 == 0, "bf16 vocab must be a multiple of 256");
   }
+  DG_ARG(m->lm_head_format == DG_LM_STORAGE || m->lm_head_format == DG_LM_E4M3, "unknown lm_head_format");
+  DG_ARG(m->n_layers >= 0 && m->n_layers <= 64, "n_layers must be in [0, 64]");
+  if (m->n_layers > 1) DG_UNSUP(m->n_experts == 0, "the MoE block needs the single-layer model");
+  if (m->lm_head_format == DG_LM_E4M3) {
+    DG_ARG(m->lm_head_scale != nullptr, "lm_head_scale is NULL");
+    DG_UNSUP(m->dtype == DG_BF16 && m->d_model % 128 == 0, "an e4m3 LM head needs bf16 and d_model % 128 == 0");
+  }
+  DG_ARG(m->expert_format == DG_LM_STORAGE || m->expert_format == DG_LM_E4M3, "unknown expert_format");
+  if (m->expert_format == DG_LM_E4M3)
+    DG_ARG(m->n_experts > 0 && m->w_gate_scale && m->w_up_scale && m->w_down_scale,
+           "e4m3 experts need n_experts > 0 and the three row-scale arrays");
   if (m->n_experts != 0) {
     DG_ARG(m->n_experts > 0 && m->top_k > 0 && m->top_k <= m->n_experts && m->moe_inter > 0 &&
                m->n_shared >= 0,
@@ -147,6 +169,62 @@ dg_status check_launch(const char* what) {
   return DG_OK;
 }
 
+// Layer l's slice of a stacked weight of `count` elements per layer.
+const void* layer_w(const dg_ctx* c, const void* base, int l, size_t count) {
+  return static_cast<const char*>(base) + (size_t)l * count * c->es;
+}
+
+// Request b's prompt K (or V) cache of layer l: [L][S_b][Hk][h] per request.
+const void* layer_prefix(const dg_ctx* c, const void* base, int b, int l) {
+  if (!base) return nullptr;
+  return static_cast<const char*>(base) + (size_t)l * c->S[b] * c->m.n_kv_heads * c->m.head_dim * c->es;
+}
+
+// Binds each layer's projection GEMMs (bf16) to the context's buffers and
+// that layer's weights: Q/K/V from xres[l], Wo + residual into xres[l + 1].
+bool prepare_layer_gemms(dg_ctx* c) {
+  const int d = c->m.d_model, qd = c->m.n_q_heads * c->m.head_dim, kd = c->m.n_kv_heads * c->m.head_dim;
+  for (int l = 0; l < c->L; ++l) {
+    const void* wqkv[3] = {layer_w(c, c->m.wq, l, (size_t)qd * d), layer_w(c, c->m.wk, l, (size_t)kd * d),
+                           layer_w(c, c->m.wv, l, (size_t)kd * d)};
+    void* oqkv[3] = {c->Q, c->Kc, c->Vc};
+    const int nqkv[3] = {qd, kd, kd};
+    const void* wo[1] = {layer_w(c, c->m.wo, l, (size_t)d * qd)};
+    void* oo[1] = {c->xres[l + 1]};
+    const int no[1] = {d};
+    float *pq = c->g_qkv[l].part, *po = c->g_wo[l].part;  // keep the bound partial buffers
+    if (!dg::gemm_tc_prepare(&c->g_qkv[l], c->xres[l], c->M, d, 3, wqkv, oqkv, nqkv, c->ex.sm_count) ||
+        !dg::gemm_tc_prepare(&c->g_wo[l], c->O, c->M, qd, 1, wo, oo, no, c->ex.sm_count))
+      return false;
+    c->g_qkv[l].part = pq;
+    c->g_wo[l].part = po;
+  }
+  return true;
+}
+
+// Each layer's attention (bf16) over that layer's prompt caches; the device
+// prompt descriptors [L][B] for the f32 path.
+dg_status prepare_layer_attention(dg_ctx* c) {
+  std::vector<dg::PrefixDesc> pd((size_t)c->L * c->B);
+  for (int l = 0; l < c->L; ++l) {
+    std::vector<const void*> pk(c->B), pv(c->B);
+    for (int b = 0; b < c->B; ++b) {
+      pk[b] = layer_prefix(c, c->pk[b], b, l);
+      pv[b] = layer_prefix(c, c->pv[b], b, l);
+      pd[(size_t)l * c->B + b] = {pk[b], pv[b], c->S[b], 0};
+    }
+    if (c->m.dtype == DG_BF16) {
+      dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
+      if (!dg::attn_tc_prepare(&c->attn[l], sh, c->Q, c->Kc, c->Vc, c->S.data(), pk.data(), pv.data(), c->O,
+                               c->attn_part_o, c->attn_part_ml, c->attn_splits))
+        return DG_ERR_CUDA;
+    }
+  }
+  DG_CUDA_RET(cudaMemcpyAsync(c->d_prefix, pd.data(), pd.size() * sizeof(dg::PrefixDesc), cudaMemcpyHostToDevice,
+                              c->ex.stream));
+  return DG_OK;
+}
+
 // The launch sequence of one denoise step (steps 1-7 of the header).
 dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) {
   const int M = c->M, d = c->m.d_model, V = c->m.vocab;
@@ -155,35 +233,46 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
   dg::Exec& ex = c->ex;
   ex.launches = 0;
   dg::launch_embed(ex, dt, c->m.embed, c->cs.tok, c->X, M, d, V);
-  if (dt == DG_BF16) {
-    dg::launch_gemm_tc(ex, c->g_qkv, nullptr);
-  } else {
-    dg::launch_linear_simple(ex, dt, c->X, c->m.wq, nullptr, c->Q, M, qd, d);
-    dg::launch_linear_simple(ex, dt, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
-    dg::launch_linear_simple(ex, dt, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
-  }
   dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
-  // inside a stream capture, only an "external" record becomes an event node
-  if (c->cur_ev_start[DG_KERNEL_ATTENTION])
-    DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start[DG_KERNEL_ATTENTION], ex.stream, cudaEventRecordExternal));
-  if (dt == DG_BF16)
-    dg::launch_attn_tc(ex, c->attn);
-  else
-    dg::launch_attention_simple(ex, dt, c->Q, c->d_prefix, c->Kc, c->Vc, c->O, sh);
-  if (c->cur_ev_stop[DG_KERNEL_ATTENTION])
-    DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_stop[DG_KERNEL_ATTENTION], ex.stream, cudaEventRecordExternal));
-  if (dt == DG_BF16)
-    dg::launch_gemm_tc(ex, c->g_wo, c->X);
-  else
-    dg::launch_linear_simple(ex, dt, c->O, c->m.wo, c->X, c->Hs, M, d, qd);
+  for (int l = 0; l < c->L; ++l) {  // layer l: xres[l] -> xres[l + 1]
+    if (dt == DG_BF16) {
+      dg::launch_gemm_tc(ex, c->g_qkv[l], nullptr);
+    } else {
+      dg::launch_linear_simple(ex, dt, c->xres[l], layer_w(c, c->m.wq, l, (size_t)qd * d), nullptr, c->Q, M, qd, d);
+      dg::launch_linear_simple(ex, dt, c->xres[l], layer_w(c, c->m.wk, l, (size_t)kd * d), nullptr, c->Kc, M, kd, d);
+      dg::launch_linear_simple(ex, dt, c->xres[l], layer_w(c, c->m.wv, l, (size_t)kd * d), nullptr, c->Vc, M, kd, d);
+    }
+    // inside a stream capture, only an "external" record becomes an event node
+    // (timed: the last layer's attention)
+    const bool timed = l == c->L - 1;
+    if (timed && c->cur_ev_start[DG_KERNEL_ATTENTION])
+      DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start[DG_KERNEL_ATTENTION], ex.stream, cudaEventRecordExternal));
+    if (dt == DG_BF16)
+      dg::launch_attn_tc(ex, c->attn[l]);
+    else
+      dg::launch_attention_simple(ex, dt, c->Q, c->d_prefix + (size_t)l * c->B, c->Kc, c->Vc, c->O, sh);
+    if (timed && c->cur_ev_stop[DG_KERNEL_ATTENTION])
+      DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_stop[DG_KERNEL_ATTENTION], ex.stream, cudaEventRecordExternal));
+    if (dt == DG_BF16)
+      dg::launch_gemm_tc(ex, c->g_wo[l], c->xres[l]);
+    else
+      dg::launch_linear_simple(ex, dt, c->O, layer_w(c, c->m.wo, l, (size_t)d * qd), c->xres[l], c->xres[l + 1],
+                               M, d, qd);
+  }
   const void* hs = c->Hs;
   if (c->m.n_experts) {
     dg::launch_moe(ex, c->moe);
     hs = c->Hs2;
   }
+  // e4m3 LM head: the residual stream is quantized first (outside the LM-head timing)
+  const bool fp8 = c->m.lm_head_format == DG_LM_E4M3;
+  if (fp8) dg::launch_quantize_rows_e4m3(ex, hs, c->hs8, c->hs8_scale, M, d);
   if (c->cur_ev_start[DG_KERNEL_LMHEAD])
     DG_CUDA_RET(cudaEventRecordWithFlags(c->cur_ev_start[DG_KERNEL_LMHEAD], ex.stream, cudaEventRecordExternal));
-  if (dt == DG_BF16)
+  if (fp8)
+    dg::launch_lmhead_tc(ex, c->tm_lm_a, c->tm_lm_b, c->lm, c->inv_temp, M, d, V, c->hs8_scale,
+                         c->m.lm_head_scale);
+  else if (dt == DG_BF16)
     dg::launch_lmhead_tc(ex, c->tm_lm_a, c->tm_lm_b, c->lm, c->inv_temp, M, d, V);
   else
     dg::launch_lmhead_simple(ex, dt, hs, c->m.lm_head, c->inv_temp, c->lm, M, d, V);
@@ -206,6 +295,10 @@ dg_status enqueue_step(dg_ctx* c, const dg_schedule& s, const dg_step_out* dbg) 
       DG_CUDA_RET(cudaMemcpyAsync(dbg->k_canvas, c->Kc, (size_t)M * kd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
     if (dbg->v_canvas)
       DG_CUDA_RET(cudaMemcpyAsync(dbg->v_canvas, c->Vc, (size_t)M * kd * c->es, cudaMemcpyDeviceToDevice, ex.stream));
+    if (dbg->layer_out)
+      for (int l = 0; l < c->L; ++l)
+        DG_CUDA_RET(cudaMemcpyAsync(static_cast<char*>(dbg->layer_out) + (size_t)l * M * d * c->es, c->xres[l + 1],
+                                    (size_t)M * d * c->es, cudaMemcpyDeviceToDevice, ex.stream));
   }
   return DG_OK;
 }
@@ -244,7 +337,10 @@ dg_status build_decode_graph(dg_ctx* c, const dg_schedule& s) {
     cudaError_t e = cudaGraphCreate(&g, 0);
     cudaGraphConditionalHandle h = 0;
     if (e == cudaSuccess) e = cudaGraphConditionalHandleCreate(&h, g, 1, cudaGraphCondAssignDefault);
-    cudaGraphNode_t reset = nullptr, loop = nullptr;
+    cudaGraphNode_t reset = nullptr, loop = nullptr, ev0 = nullptr, ev1 = nullptr;
+    const cudaEvent_t t_start = c->ev_start[DG_KERNEL_DECODE].empty() ? nullptr : c->ev_start[DG_KERNEL_DECODE][0];
+    const cudaEvent_t t_stop = c->ev_stop[DG_KERNEL_DECODE].empty() ? nullptr : c->ev_stop[DG_KERNEL_DECODE][0];
+    if (e == cudaSuccess && t_start) e = cudaGraphAddEventRecordNode(&ev0, g, nullptr, 0, t_start);
     if (e == cudaSuccess) {
       cudaMemsetParams mp = {};
       mp.dst = c->cs.loop_iter;
@@ -253,7 +349,7 @@ dg_status build_decode_graph(dg_ctx* c, const dg_schedule& s) {
       mp.width = 1;
       mp.height = 1;
       mp.pitch = 4;
-      e = cudaGraphAddMemsetNode(&reset, g, nullptr, 0, &mp);
+      e = cudaGraphAddMemsetNode(&reset, g, ev0 ? &ev0 : nullptr, ev0 ? 1 : 0, &mp);
     }
     cudaGraphNodeParams cp = {};
     if (e == cudaSuccess) {
@@ -263,6 +359,7 @@ dg_status build_decode_graph(dg_ctx* c, const dg_schedule& s) {
       cp.conditional.size = 1;
       e = cudaGraphAddNode(&loop, g, &reset, 1, &cp);
     }
+    if (e == cudaSuccess && t_stop) e = cudaGraphAddEventRecordNode(&ev1, g, &loop, 1, t_stop);
     dg_status st = DG_OK;
     if (e == cudaSuccess) {
       cudaGraph_t body = cp.conditional.phGraph_out[0];
@@ -392,7 +489,7 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   dg_status st = validate_model(model);
   if (st != DG_OK) return st;
   DG_ARG(batch >= 1 && batch <= 4096, "batch must be in [1, 4096]");
-  DG_ARG(canvas_len >= 1 && canvas_len <= 256, "canvas_len must be in [1, 256]");
+  DG_ARG(canvas_len >= 1 && canvas_len <= 1024, "canvas_len must be in [1, 1024]");
   if (model->n_experts) DG_UNSUP(batch * canvas_len <= 256, "the MoE FFN needs batch * canvas_len <= 256");
   DG_ARG(prefix_len && seeds, "prefix_len / seeds is NULL");
   for (int b = 0; b < batch; ++b) {
@@ -410,6 +507,10 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   c->C = canvas_len;
   c->M = batch * canvas_len;
   c->es = model->dtype == DG_F32 ? 4 : 2;
+  c->L = std::max(1, (int)model->n_layers);
+  c->g_qkv.resize(c->L);
+  c->g_wo.resize(c->L);
+  c->attn.resize(c->L);
   c->inv_temp = inv_temp;
   c->ex.stream = static_cast<cudaStream_t>(cuda_stream);
   for (int b = 0; b < batch; ++b) {
@@ -427,7 +528,7 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   }
   if (model->dtype == DG_BF16) {
     c->lm.P = dg::lmhead_tc_partitions(c->M, model->vocab, c->ex.sm_count);
-    c->attn_splits = dg::attn_tc_splits(batch, canvas_len, model->n_q_heads, c->S.data(), c->ex.sm_count);
+    c->attn_splits = dg::attn_tc_splits(batch, canvas_len, model->n_q_heads, model->n_kv_heads, c->S.data(), c->ex.sm_count);
     c->attn_splits_cap = c->attn_splits;
     // tile / split choice only (buffers are bound after the workspace exists)
     const int qd = model->n_q_heads * model->head_dim, kd = model->n_kv_heads * model->head_dim;
@@ -436,8 +537,8 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
     const int nqkv[3] = {qd, kd, kd};
     const void* wo[1] = {model->wo};
     const int no[1] = {model->d_model};
-    if (!dg::gemm_tc_prepare(&c->g_qkv, model->embed, c->M, model->d_model, 3, wqkv, none, nqkv, c->ex.sm_count) ||
-        !dg::gemm_tc_prepare(&c->g_wo, model->embed, c->M, qd, 1, wo, none, no, c->ex.sm_count))
+    if (!dg::gemm_tc_prepare(&c->g_qkv[0], model->embed, c->M, model->d_model, 3, wqkv, none, nqkv, c->ex.sm_count) ||
+        !dg::gemm_tc_prepare(&c->g_wo[0], model->embed, c->M, qd, 1, wo, none, no, c->ex.sm_count))
       return fail(DG_ERR_CUDA);
   }
   else
@@ -459,40 +560,26 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   layout_workspace(c, c->ws, &total);
   c->ex.err = c->err;
   if (model->dtype == DG_BF16) {
-    const int qd = model->n_q_heads * model->head_dim, kd = model->n_kv_heads * model->head_dim;
-    const void* wqkv[3] = {model->wq, model->wk, model->wv};
-    void* oqkv[3] = {c->Q, c->Kc, c->Vc};
-    const int nqkv[3] = {qd, kd, kd};
-    const void* wo[1] = {model->wo};
-    void* oo[1] = {c->Hs};
-    const int no[1] = {model->d_model};
-    dg::GemmTc gq = c->g_qkv, gw = c->g_wo;  // keep the bound buffers
-    const void* lm_in = model->n_experts ? c->Hs2 : c->Hs;
+    const bool fp8 = model->lm_head_format == DG_LM_E4M3;
+    const void* lm_in = fp8 ? (const void*)c->hs8 : model->n_experts ? c->Hs2 : c->Hs;
     if (!dg::lmhead_tc_prepare(lm_in, model->lm_head, c->M, model->d_model, model->vocab, &c->tm_lm_a,
-                               &c->tm_lm_b) ||
-        !dg::gemm_tc_prepare(&c->g_qkv, c->X, c->M, model->d_model, 3, wqkv, oqkv, nqkv, c->ex.sm_count) ||
-        !dg::gemm_tc_prepare(&c->g_wo, c->O, c->M, qd, 1, wo, oo, no, c->ex.sm_count))
-      return fail(DG_ERR_CUDA);
-    c->g_qkv.part = gq.part;
-    c->g_wo.part = gw.part;
-    dg::AttnShape sh{batch, canvas_len, model->n_q_heads, model->n_kv_heads, model->head_dim};
-    if (!dg::attn_tc_prepare(&c->attn, sh, c->Q, c->Kc, c->Vc, c->S.data(), c->pk.data(), c->pv.data(), c->O,
-                             c->attn.part_o, c->attn.part_ml, c->attn_splits))
+                               &c->tm_lm_b, fp8) ||
+        !prepare_layer_gemms(c))
       return fail(DG_ERR_CUDA);
     if (model->n_experts) {
-      dg::MoeShape ms{c->M, model->d_model, model->n_experts, model->top_k, model->n_shared, model->moe_inter};
+      dg::MoeShape ms{c->M, model->d_model, model->n_experts, model->top_k, model->n_shared, model->moe_inter,
+                      model->expert_format == DG_LM_E4M3};
+      const float* scales[3] = {model->w_gate_scale, model->w_up_scale, model->w_down_scale};
       if (!dg::moe_prepare(&c->moe, ms, c->Hs, c->Hs2, model->w_router, model->w_gate, model->w_up, model->w_down,
-                           c->moe_ws, c->ex.sm_count))
+                           c->moe_ws, c->ex.sm_count, scales))
         return fail(DG_ERR_UNSUPPORTED);
     }
   }
 
-  std::vector<dg::PrefixDesc> pd(batch);
-  for (int b = 0; b < batch; ++b) pd[b] = {c->pk[b], c->pv[b], c->S[b], 0};
-  std::vector<uint32_t> zeros(batch + 1, 0);
+  st = prepare_layer_attention(c);
+  if (st != DG_OK) return fail(st);
   cudaStream_t sm = c->ex.stream;
-  if (cudaMemcpyAsync(c->d_prefix, pd.data(), batch * sizeof(dg::PrefixDesc), cudaMemcpyHostToDevice, sm) != cudaSuccess ||
-      cudaMemcpyAsync(c->cs.seed, seeds, batch * sizeof(uint64_t), cudaMemcpyHostToDevice, sm) != cudaSuccess ||
+  if (cudaMemcpyAsync(c->cs.seed, seeds, batch * sizeof(uint64_t), cudaMemcpyHostToDevice, sm) != cudaSuccess ||
       cudaMemsetAsync(c->cs.counters, 0, (batch + 1) * sizeof(uint32_t), sm) != cudaSuccess ||
       cudaMemsetAsync(c->err, 0, sizeof(int32_t), sm) != cudaSuccess) {
     set_last_error("initial copies failed");
@@ -552,13 +639,14 @@ dg_status dg_canvas_reset_fixed(dg_ctx* ctx, const uint64_t* seeds, const uint8_
 dg_status dg_canvas_block_kv(dg_ctx* c, void* k_out, void* v_out) {
   DG_ARG(c != nullptr, "ctx is NULL");
   DG_ARG(k_out && v_out, "k_out / v_out is NULL");
+  DG_UNSUP(c->L == 1, "block K/V need the single-layer model (deeper stacks need a causal encoder pass)");
   const int M = c->M, d = c->m.d_model, V = c->m.vocab;
   const int qd = c->m.n_q_heads * c->m.head_dim, kd = c->m.n_kv_heads * c->m.head_dim;
   dg::Exec& ex = c->ex;
   ex.launches = 0;
   dg::launch_embed(ex, c->m.dtype, c->m.embed, c->cs.tok, c->X, M, d, V);
   if (c->m.dtype == DG_BF16) {
-    dg::launch_gemm_tc(ex, c->g_qkv, nullptr);
+    dg::launch_gemm_tc(ex, c->g_qkv[0], nullptr);
   } else {
     dg::launch_linear_simple(ex, c->m.dtype, c->X, c->m.wk, nullptr, c->Kc, M, kd, d);
     dg::launch_linear_simple(ex, c->m.dtype, c->X, c->m.wv, nullptr, c->Vc, M, kd, d);
@@ -591,19 +679,11 @@ dg_status dg_canvas_set_prefix(dg_ctx* c, const int32_t* prefix_len, const void*
     c->pv[b] = prefix_len[b] ? prefix_v[b] : nullptr;
     c->max_S = std::max(c->max_S, (int)prefix_len[b]);
   }
-  if (c->m.dtype == DG_BF16) {
-    // the split partial buffers were sized at init: never exceed that split count
-    c->attn_splits =
-        std::min(c->attn_splits_cap, dg::attn_tc_splits(c->B, c->C, c->m.n_q_heads, c->S.data(), c->ex.sm_count));
-    dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
-    if (!dg::attn_tc_prepare(&c->attn, sh, c->Q, c->Kc, c->Vc, c->S.data(), c->pk.data(), c->pv.data(), c->O,
-                             c->attn.part_o, c->attn.part_ml, c->attn_splits))
-      return DG_ERR_CUDA;
-  }
-  std::vector<dg::PrefixDesc> pd(c->B);
-  for (int b = 0; b < c->B; ++b) pd[b] = {c->pk[b], c->pv[b], c->S[b], 0};
-  DG_CUDA_RET(cudaMemcpyAsync(c->d_prefix, pd.data(), c->B * sizeof(dg::PrefixDesc), cudaMemcpyHostToDevice,
-                              c->ex.stream));
+  if (c->m.dtype == DG_BF16)  // the split partial buffers were sized at init: never exceed that split count
+    c->attn_splits = std::min(c->attn_splits_cap, dg::attn_tc_splits(c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads,
+                                                                    c->S.data(), c->ex.sm_count));
+  dg_status st = prepare_layer_attention(c);
+  if (st != DG_OK) return st;
   DG_CUDA_RET(cudaStreamSynchronize(c->ex.stream));
   return DG_OK;
 }
@@ -623,14 +703,12 @@ dg_status dg_decode_block(dg_ctx* ctx, const dg_schedule* sched, int32_t* tokens
     if (st != DG_OK) return st;
     DG_CUDA_RET(cudaGraphLaunch(ctx->decode_graph, ctx->ex.stream));
   }
-  st = read_device_error(ctx);
-  if (st != DG_OK) return st;
+  // results and the device error word come back together: one wait
   if (tokens_out)
     DG_CUDA_RET(cudaMemcpyAsync(tokens_out, ctx->cs.tok, ctx->M * sizeof(int32_t), cudaMemcpyDefault, ctx->ex.stream));
   if (steps_out)
     DG_CUDA_RET(cudaMemcpyAsync(steps_out, ctx->cs.step, ctx->B * sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->ex.stream));
-  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
-  return DG_OK;
+  return read_device_error(ctx);
 }
 
 dg_status dg_canvas_get_state(dg_ctx* ctx, dg_state* h) {
@@ -668,8 +746,10 @@ dg_status dg_canvas_set_state(dg_ctx* ctx, const dg_state* h) {
 dg_status dg_canvas_set_kernel_timing(dg_ctx* ctx, int32_t kernel, int32_t n, void* const* starts,
                                       void* const* stops) {
   DG_ARG(ctx != nullptr, "ctx is NULL");
-  DG_ARG(kernel == DG_KERNEL_LMHEAD || kernel == DG_KERNEL_ATTENTION, "unknown kernel id");
+  DG_ARG(kernel == DG_KERNEL_LMHEAD || kernel == DG_KERNEL_ATTENTION || kernel == DG_KERNEL_DECODE,
+         "unknown kernel id");
   DG_ARG(n >= 0 && n <= 64, "n must be in [0, 64]");
+  DG_ARG(kernel != DG_KERNEL_DECODE || n <= 1, "the decode loop takes one event pair");
   if (n > 0) DG_ARG(starts && stops, "event arrays are NULL");
   for (int i = 0; i < n; ++i) DG_ARG(starts[i] && stops[i], "NULL event");
   DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));

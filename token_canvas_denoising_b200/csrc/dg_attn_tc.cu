@@ -7,27 +7,36 @@
 // own K/V are recomputed every step (架构解剖 2). Per query head q (KV head
 // g = q / (Hq/Hk)): O = softmax(Q K^T / sqrt(h)) V over [prefix keys; canvas keys].
 //
-// CTA work item: (request b, query head q, 128-query tile, KV split). The KV
-// sequence is walked in 128-key tiles (prefix tiles from the request's own
-// tensor map, then canvas tiles) through 3-slot TMA rings for K and for V.
-//   warp 0   : TMA producer: Q once; K tiles one ahead of V tiles (a K slot
-//              frees when its QK completes, a V slot when its PV does);
-//              prompt-prefix tiles a few tiles ahead are prefetched into L2
-//   warp 1   : TMEM allocator and MMA issuer: S_j = Q K_j^T (M=N=128, K=128)
-//              into one of two TMEM score buffers, then O += P_j V_j (V as an
-//              MN-major operand) into the TMEM output accumulator. Q and P are
-//              A operands read from TMEM, so shared memory only feeds K and V
-//              (the tile's operand traffic through shared memory halves).
-//   warps 2-5: softmax, one query row per thread: copy the Q row from shared
-//              memory into TMEM once; per tile read S_j from TMEM, mask the
-//              keys past the tile's end, exponentiate in base 2 against a
-//              running maximum, write P_j (bf16 pairs) into TMEM. The running
-//              maximum is only raised when the tile's maximum exceeds it by
-//              more than 8 (a factor 256), and then O and the running sum are
-//              rescaled in place; otherwise the stale maximum is kept (the
-//              result is the same ratio). The decision is per warp, since the
-//              TMEM accesses are collective.
-// TMEM columns: S0 [0,128) | S1 [128,256) | O [256,384) | Q [384,448) | P [448,512).
+// CTA work item: two 128-query tiles ("slots" A and B) that read the same KV
+// head of the same request -- the two query tiles of one head, or the same
+// tile of two heads of one KV group -- and one KV split. The KV sequence is
+// walked once, in 128-key tiles (prefix tiles from the request's own tensor
+// map, then canvas tiles), through a 3-slot K ring and a 2-slot V ring; every
+// K and V tile feeds both slots' MMAs, so a tile crosses L2 -> SM once for
+// 256 queries.
+//   warp 0   : TMA producer: Q_A and Q_B once; K tiles one ahead of V tiles
+//              (a K slot frees when both slots' QK are done, a V slot when
+//              both PVs are); prompt tiles a few ahead are prefetched into L2
+//   warp 1   : TMEM allocator and MMA issuer. Per key tile j, in this order:
+//              PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j), where QK_x(j) is
+//              S_x = Q_x K_j^T (M = N = 128, K = 128) and PV_x(j) is
+//              O_x += P_x V_j with P_x read from tensor memory (V as an
+//              MN-major operand). tcgen05.mma ops of one thread execute in
+//              issue order, so QK_x(j) may overwrite the columns PV_x(j-1)
+//              reads P_x from, and the commit after QK_x(j) also covers
+//              PV_x(j-1).
+//   warps 2-5: softmax of slot A, warps 6-9: softmax of slot B, one query
+//              row per thread: read S_x from TMEM, mask keys past the tile's
+//              end, exponentiate in base 2 against a running maximum, write
+//              P_x (bf16 pairs) over the first 64 columns of S_x. While one
+//              slot's warps exponentiate, the tensor core runs the other
+//              slot's MMAs, so the MUFU and the tensor pipe stay busy
+//              together. The running maximum is raised only when the tile's
+//              maximum exceeds it by more than 8 (a factor 256), and then O_x
+//              and the running sum are rescaled in place; the decision is per
+//              warp, since the TMEM accesses are warp-collective.
+// TMEM columns: S_A [0,128) | S_B [128,256) | O_A [256,384) | O_B [384,512);
+// P_x occupies columns [0,64) of S_x.
 // With one split the rows are normalised and stored as bf16; with several,
 // unnormalised O and (max, sum) go to a partial buffer for attn_merge_kernel.
 #include <cstring>
@@ -41,24 +50,27 @@ namespace attntc {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kTile = 128;
 constexpr int kAtom = 128 * 128;       // 128 rows x 128 B = 16 KB
 constexpr int kMatBytes = 2 * kAtom;   // a 128 x 128 bf16 tile = 32 KB
-constexpr int kSlots = 3;              // K ring and V ring depth
-// smem: Q | K0 K1 K2 | V0 V1 V2 | barriers. The dynamic shared window starts
-// 1024-aligned (after the CTA's reserved 1 KB); the kernel checks this
+constexpr int kKSlots = 3;             // K ring depth
+constexpr int kVSlots = 2;             // V ring depth
+// smem: Q_A Q_B | K0 K1 K2 | V0 V1 | barriers. The dynamic shared window
+// starts 1024-aligned (after the CTA's reserved 1 KB); the kernel checks this
 // instead of reserving alignment slack.
 constexpr int kOffQ = 0;
-constexpr int kOffK = kMatBytes;
-constexpr int kOffV = kOffK + kSlots * kMatBytes;
-constexpr int kOffBar = kOffV + kSlots * kMatBytes;
+constexpr int kOffK = 2 * kMatBytes;
+constexpr int kOffV = kOffK + kKSlots * kMatBytes;
+constexpr int kOffBar = kOffV + kVSlots * kMatBytes;
 constexpr int kSmemBytes = kOffBar + 256;
 static_assert(kSmemBytes <= 232448, "attention tile exceeds the opt-in shared memory of a CTA");
 constexpr int kMaxReq = 8;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 constexpr int kAhead = 4;                 // prompt-prefix tiles prefetched into L2 ahead of their load
-constexpr uint32_t kColO = 256, kColQ = 384, kColP = 448;
+// TMEM column of slot x's scores (and P) and of its output accumulator
+__host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
+__host__ __device__ constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * 128u; }
 
 struct Maps {
   CUtensorMap q;    // [B*C][Hq*h]
@@ -72,7 +84,10 @@ struct Params {
   int b0, nreq;  // requests [b0, b0 + nreq) in this launch
   int C, Hq, Hk;
   int S[kMaxReq];
-  int q_tiles, splits;
+  int q_tiles;       // 128-query tiles per canvas
+  int items;         // (head, query tile) pairs per (request, KV head) = (Hq/Hk) * q_tiles
+  int pairs;         // CTAs per (request, KV head, split) = ceil(items / 2)
+  int splits;
   int rows_total;    // B_total * C * Hq (partial buffer row count)
   float scale_log2;  // log2(e) / sqrt(h)
   __nv_bfloat16* O;  // [B*C][Hq*h]
@@ -94,26 +109,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
   uint8_t* smem = smem_raw;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* q_full = bar + 0;      // Q tile landed in shared memory
-  uint64_t* q_tmem = bar + 1;      // Q copied into TMEM (4 softmax warps)
-  uint64_t* k_full = bar + 2;      // [3]
-  uint64_t* v_full = bar + 5;      // [3]
-  uint64_t* k_empty = bar + 8;     // [3] QK_i done: K slot i % 3 free
-  uint64_t* v_empty = bar + 11;    // [3] PV_i done: V slot i % 3 free
-  uint64_t* s_full = bar + 14;     // [2] S_i in TMEM buffer i & 1
-  uint64_t* s_free = bar + 16;     // [2] S buffer read by the softmax (4 warps)
-  uint64_t* p_full = bar + 18;     // P_i in TMEM (4 warps)
-  uint64_t* pv_done = bar + 19;    // PV_i complete: O stable, P columns free
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 20);
+  uint64_t* q_full = bar + 0;                   // [2] Q_x landed
+  uint64_t* k_full = bar + 2;                   // [3]
+  uint64_t* k_empty = k_full + kKSlots;         // [3] the last slot's QK of the tile done
+  uint64_t* v_full = k_empty + kKSlots;         // [2]
+  uint64_t* v_empty = v_full + kVSlots;         // [2] the last slot's PV of the tile done
+  uint64_t* s_full = v_empty + kVSlots;         // [2] S_x in TMEM (and PV_x of the previous tile done)
+  uint64_t* p_full = s_full + 2;                // [2] P_x in TMEM (4 warps)
+  uint64_t* pv_done = p_full + 2;               // [2] every MMA of slot x done (end of the walk)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % p.q_tiles;
-  const int qh = blockIdx.x / p.q_tiles;
+  const int g = blockIdx.x / p.pairs;          // KV head
+  const int pair = blockIdx.x % p.pairs;
+  const int nslots = min(2, p.items - 2 * pair);
+  // (query head, query tile) of slot x; slot B repeats A's when it is unused
+  auto slot_head = [&](int x) { return g * (p.Hq / p.Hk) + min(2 * pair + x, p.items - 1) / p.q_tiles; };
+  auto slot_tile = [&](int x) { return min(2 * pair + x, p.items - 1) % p.q_tiles; };
   const int lb = blockIdx.y;            // request within this launch
   const int b = p.b0 + lb;              // request index
   const int z = blockIdx.z;             // KV split
-  const int g = qh / (p.Hq / p.Hk);
   const int S = p.S[lb];
   const int nps = (S + kTile - 1) / kTile;
   const int nct = (p.C + kTile - 1) / kTile;
@@ -123,20 +139,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int n = t1 - t0;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_tmem, 4);
-    for (int i = 0; i < kSlots; ++i) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
+    for (int i = 0; i < kKSlots; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
+      mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-    }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -171,17 +187,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const CUtensorMap *mk, *mv;
         int y;
         tile_src(i, mk, mv, y);
-        uint8_t* kb = smem + kOffK + (i % kSlots) * kMatBytes;
-        mbar_arrive_expect_tx(&k_full[i % kSlots], kMatBytes);
-        tma_load_3d(kb, mk, &k_full[i % kSlots], 0, y, g * 2, pol);
+        mbar_arrive_expect_tx(&k_full[i % kKSlots], kMatBytes);
+        tma_load_3d(smem + kOffK + (i % kKSlots) * kMatBytes, mk, &k_full[i % kKSlots], 0, y, g * 2, pol);
       };
       auto load_v = [&](int i) {
         const CUtensorMap *mk, *mv;
         int y;
         tile_src(i, mk, mv, y);
-        uint8_t* vb = smem + kOffV + (i % kSlots) * kMatBytes;
-        mbar_arrive_expect_tx(&v_full[i % kSlots], kMatBytes);
-        tma_load_3d(vb, mv, &v_full[i % kSlots], 0, y, g * 2, pol);
+        mbar_arrive_expect_tx(&v_full[i % kVSlots], kMatBytes);
+        tma_load_3d(smem + kOffV + (i % kVSlots) * kMatBytes, mv, &v_full[i % kVSlots], 0, y, g * 2, pol);
       };
       // prompt-prefix tiles further ahead are pulled into L2 early
       auto prefetch = [&](int i) {
@@ -193,131 +207,116 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       int nk = 0, nv = 0;  // next K tile and next V tile to load
       // the prompt prefix is an input of the step: its first tiles may be
       // fetched before the predecessor kernels are done
-      while (nk < kSlots && nk < n && t0 + nk < nps) {
-        load_k(nk);
-        load_v(nk);
-        ++nk;
-        ++nv;
-      }
+      while (nk < kKSlots && nk < n && t0 + nk < nps) load_k(nk++);
+      while (nv < kVSlots && nv < n && t0 + nv < nps) load_v(nv++);
       for (int i = nk; i < nk + kAhead; ++i) prefetch(i);
       griddep_wait();
-      mbar_arrive_expect_tx(q_full, kMatBytes);
-      tma_load_3d(smem + kOffQ, &maps.q, q_full, 0, b * p.C + qt * kTile, qh * 2, pol);
-      // K runs one tile ahead of V
+      for (int x = 0; x < nslots; ++x) {
+        mbar_arrive_expect_tx(&q_full[x], kMatBytes);
+        tma_load_3d(smem + kOffQ + x * kMatBytes, &maps.q, &q_full[x], 0, b * p.C + slot_tile(x) * kTile,
+                    slot_head(x) * 2, pol);
+      }
+      // K runs one tile ahead of V (the MMA order is PV(j-1) then QK(j))
       while (nv < n && !*abort_flag) {
         if (nk < n && nk <= nv + 1) {
-          if (nk >= kSlots && !mbar_wait(&k_empty[nk % kSlots], ((nk / kSlots) - 1) & 1, p.err, abort_flag)) break;
+          if (nk >= kKSlots &&
+              !mbar_wait(&k_empty[nk % kKSlots], ((nk / kKSlots) - 1) & 1, p.err, abort_flag))
+            break;
           load_k(nk);
           prefetch(nk + kAhead);
           ++nk;
         } else {
-          if (nv >= kSlots && !mbar_wait(&v_empty[nv % kSlots], ((nv / kSlots) - 1) & 1, p.err, abort_flag)) break;
+          if (nv >= kVSlots &&
+              !mbar_wait(&v_empty[nv % kVSlots], ((nv / kVSlots) - 1) & 1, p.err, abort_flag))
+            break;
           load_v(nv);
           ++nv;
         }
       }
-      if (*abort_flag) {  // drain this CTA's own copies: the last load of each slot
-        mbar_wait(q_full, 0, p.err, nullptr);
-        for (int i = nk - kSlots; i < nk; ++i)
-          if (i >= 0) mbar_wait(&k_full[i % kSlots], (i / kSlots) & 1, p.err, nullptr);
-        for (int i = nv - kSlots; i < nv; ++i)
-          if (i >= 0) mbar_wait(&v_full[i % kSlots], (i / kSlots) & 1, p.err, nullptr);
+      if (*abort_flag) {  // drain this CTA's own copies: Q and the last load of each slot
+        for (int x = 0; x < nslots; ++x) mbar_wait(&q_full[x], 0, p.err, nullptr);
+        for (int i = nk - kKSlots; i < nk; ++i)
+          if (i >= 0) mbar_wait(&k_full[i % kKSlots], (i / kKSlots) & 1, p.err, nullptr);
+        for (int i = nv - kVSlots; i < nv; ++i)
+          if (i >= 0) mbar_wait(&v_full[i % kVSlots], (i / kVSlots) & 1, p.err, nullptr);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    griddep_wait();
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(128, 128, false);
       const uint32_t id_pv = idesc_bf16_f32(128, 128, true);
-      bool ok = mbar_wait(q_tmem, 0, p.err, abort_flag);
-      auto issue_qk = [&](int i) -> bool {
-        const int s = i & 1, slot = i % kSlots;
-        if (!mbar_wait(&k_full[slot], (i / kSlots) & 1, p.err, abort_flag)) return false;
-        if (i >= 2 && !mbar_wait(&s_free[s], ((i >> 1) - 1) & 1, p.err, abort_flag)) return false;
+      bool ok = true;
+      for (int x = 0; ok && x < nslots; ++x) ok = mbar_wait(&q_full[x], 0, p.err, abort_flag);
+      auto qk = [&](int x, int i) -> bool {
+        const int slot = i % kKSlots;
+        if (x == 0 && !mbar_wait(&k_full[slot], (i / kKSlots) & 1, p.err, abort_flag)) return false;
         tc_fence_after();
+        const uint32_t qbase = smem_u32(smem + kOffQ + x * kMatBytes);
         const uint32_t kbase = smem_u32(smem + kOffK + slot * kMatBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + s * 128, tmem + kColQ + kk * 8, kdesc(kbase, kk), id_qk, kk != 0);
-        mma_commit(&s_full[s]);
-        mma_commit(&k_empty[slot]);
+          mma_bf16_ss(tmem + col_s(x), kdesc(qbase, kk), kdesc(kbase, kk), id_qk, kk != 0);
+        mma_commit(&s_full[x]);
+        if (x == nslots - 1) mma_commit(&k_empty[slot]);
         return true;
       };
-      if (ok && n > 0) ok = issue_qk(0);
-      for (int i = 0; ok && i < n; ++i) {
-        if (i + 1 < n && !(ok = issue_qk(i + 1))) break;
-        const int slot = i % kSlots;
-        if (!mbar_wait(p_full, i & 1, p.err, abort_flag)) break;
-        if (!mbar_wait(&v_full[slot], (i / kSlots) & 1, p.err, abort_flag)) break;
+      auto pv = [&](int x, int i) -> bool {
+        const int slot = i % kVSlots;
+        if (!mbar_wait(&p_full[x], i & 1, p.err, abort_flag)) return false;
+        if (x == 0 && !mbar_wait(&v_full[slot], (i / kVSlots) & 1, p.err, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vbase = smem_u32(smem + kOffV + slot * kMatBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, umma_desc_sw128(vbase + kk * 2048, kAtom, 1024), id_pv,
-                      (i | kk) != 0);
-        mma_commit(pv_done);
-        mma_commit(&v_empty[slot]);
+          mma_bf16_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8, umma_desc_sw128(vbase + kk * 2048, kAtom, 1024),
+                      id_pv, (i | kk) != 0);
+        if (x == nslots - 1) mma_commit(&v_empty[slot]);
+        return true;
+      };
+      for (int x = 0; ok && n > 0 && x < nslots; ++x) ok = qk(x, 0);
+      for (int i = 0; ok && i < n; ++i) {
+        for (int x = 0; ok && x < nslots; ++x) {
+          ok = pv(x, i);
+          if (ok && i + 1 < n) ok = qk(x, i + 1);
+        }
       }
+      // every MMA of the walk has landed in O before the epilogue reads it
+      for (int x = 0; x < nslots; ++x) mma_commit(&pv_done[x]);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    griddep_wait();
+    const int x = (warp - 2) >> 2;  // slot of this warpgroup
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // query row within the tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t s_col = col_s(x), o_col = col_o(x);
     float m_run = -INFINITY, l = 0.f;
-    // Q row into TMEM columns [384, 448): 16-byte chunk c of swizzle atom a
-    // holds head dims a*64 + c*8 .. +7, i.e. columns a*32 + c*4 .. +3
-    bool ok = mbar_wait_warp(q_full, 0, p.err, abort_flag);
-    if (ok) {
-      const uint8_t* qrow = smem + kOffQ + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-      for (int a = 0; a < 2; ++a) {
-        uint32_t u[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(qrow + a * kAtom + ((c ^ (r & 7)) << 4));
-          u[c * 4 + 0] = v.x;
-          u[c * 4 + 1] = v.y;
-          u[c * 4 + 2] = v.z;
-          u[c * 4 + 3] = v.w;
-        }
-        tmem_st32(tmem + lane_off + kColQ + a * 32, u);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_tmem);
-    }
+    bool ok = x < nslots;
     for (int i = 0; ok && i < n; ++i) {
-      const int s = i & 1;
-      if (!(ok = mbar_wait_warp(&s_full[s], (i >> 1) & 1, p.err, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(&s_full[x], i & 1, p.err, abort_flag))) break;
       tc_fence_after();
-      float x[128];
+      float v[128];
       {
         uint32_t u[128];
-        tmem_ld128_sync(tmem + lane_off + s * 128, u);
+        tmem_ld128_sync(tmem + lane_off + s_col, u);
 #pragma unroll
-        for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 128; ++e) v[e] = __uint_as_float(u[e]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[s]);
       // keys of this tile that exist
       const int j = t0 + i;
       const int valid = (j < nps) ? min(kTile, S - j * kTile) : min(kTile, p.C - (j - nps) * kTile);
       if (valid < kTile) {  // ragged last tile (uniform over the CTA)
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (c >= valid) x[c] = -INFINITY;
+          if (c >= valid) v[c] = -INFINITY;
       }
       // row maximum over 8 independent chains (short dependency chains)
       float mx[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = x[c];
+      for (int c = 0; c < 8; ++c) mx[c] = v[c];
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
 #pragma unroll
       for (int w = 4; w > 0; w >>= 1)
 #pragma unroll
@@ -334,33 +333,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         alpha = ex2_approx(m_run - m_new);
         m_run = m_new;
       }
-      // P = 2^(x scale - m_run) as bf16 pairs, row sum over 8 chains
+      // P = 2^(s scale - m_run) as bf16 pairs, row sum over 8 chains
       uint32_t pk[64];
       float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       const float neg_m = -m_run;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(x[2 * c], p.scale_log2, neg_m));
-        const float p1 = ex2_approx(fmaf(x[2 * c + 1], p.scale_log2, neg_m));
+        const float p0 = ex2_approx(fmaf(v[2 * c], p.scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(v[2 * c + 1], p.scale_log2, neg_m));
         ls[(2 * c) & 7] += p0;
         ls[(2 * c + 1) & 7] += p1;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-      // PV_{i-1} complete: O holds it (for the rescale) and the P columns are free
-      if (i > 0) {
-        if (!(ok = mbar_wait_warp(pv_done, (i - 1) & 1, p.err, abort_flag))) break;
-        tc_fence_after();
-      }
+      // s_full(i) was committed after PV_x(i-1): O_x holds it and may be rescaled
       if (rescale && i > 0) {
         l *= alpha;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t u[32];
-          tmem_ld32_sync(tmem + lane_off + kColO + c * 32, u);
+          tmem_ld32_sync(tmem + lane_off + o_col + c * 32, u);
 #pragma unroll
           for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-          tmem_st32(tmem + lane_off + kColO + c * 32, u);
+          tmem_st32(tmem + lane_off + o_col + c * 32, u);
         }
       }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
@@ -368,30 +363,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         uint32_t u[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) u[e] = pk[e];
-        tmem_st32(tmem + lane_off + kColP, u);
+        tmem_st32(tmem + lane_off + s_col, u);
 #pragma unroll
         for (int e = 0; e < 32; ++e) u[e] = pk[32 + e];
-        tmem_st32(tmem + lane_off + kColP + 32, u);
+        tmem_st32(tmem + lane_off + s_col + 32, u);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[x]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n > 0 && mbar_wait_warp(pv_done, (n - 1) & 1, p.err, abort_flag)) {
+    if (ok && n > 0 && mbar_wait_warp(&pv_done[x], 0, p.err, abort_flag)) {
       tc_fence_after();
-      const int qrow = qt * kTile + r;
+      const int qrow = slot_tile(x) * kTile + r;
       const bool has_row = qrow < p.C;
       const size_t grow = (size_t)(b * p.C + qrow);
       const float inv = 1.f / l;
+      const int q = slot_head(x);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t u[32];
-        tmem_ld32_sync(tmem + lane_off + kColO + c * 32, u);
+        tmem_ld32_sync(tmem + lane_off + o_col + c * 32, u);
         if (!has_row) continue;
         if (p.splits == 1) {
-          uint4* dst = reinterpret_cast<uint4*>(p.O + grow * p.Hq * 128 + qh * 128 + c * 32);
+          uint4* dst = reinterpret_cast<uint4*>(p.O + grow * p.Hq * 128 + q * 128 + c * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 w;
@@ -403,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             dst[v4] = w;
           }
         } else {
-          const size_t prow_i = (size_t)z * p.rows_total + grow * p.Hq + qh;
+          const size_t prow_i = (size_t)z * p.rows_total + grow * p.Hq + q;
           float4* dst = reinterpret_cast<float4*>(p.part_o + prow_i * 128 + c * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 8; ++v4)
@@ -453,14 +449,20 @@ __global__ void attn_merge_kernel(const float* __restrict__ part_o, const float*
   dst[1] = __floats2bfloat162_rn(o2 * inv, o3 * inv);
 }
 
+// CTAs per (request, KV split): KV heads x pairs of (head, query tile).
+int attn_ctas_per_request(int C, int Hq, int Hk) {
+  const int items = (Hq / Hk) * ceil_div(C, kTile);
+  return Hk * ceil_div(items, 2);
+}
+
 }  // namespace attntc
 
 // ---------------------------------------------------------------- host side
-int attn_tc_splits(int B, int C, int Hq, const int* S, int sm_count) {
+int attn_tc_splits(int B, int C, int Hq, int Hk, const int* S, int sm_count) {
   const int q_tiles = ceil_div(C, 128);
   int min_tiles = 1 << 30;
   for (int b = 0; b < B; ++b) min_tiles = std::min(min_tiles, ceil_div(S[b], 128) + q_tiles);
-  int splits = sm_count / std::max(1, B * Hq * q_tiles);
+  int splits = sm_count / std::max(1, B * attntc::attn_ctas_per_request(C, Hq, Hk));
   splits = std::max(1, std::min(splits, std::min(min_tiles, 16)));
   return splits;
 }
@@ -518,6 +520,8 @@ void launch_attn_tc(Exec& ex, const AttnTc& at) {
   const AttnShape& sh = at.sh;
   const int q_tiles = ceil_div(sh.C, 128);
   const int rows_total = sh.B * sh.C * sh.Hq;
+  const int items = (sh.Hq / sh.Hk) * q_tiles;
+  const int pairs = ceil_div(items, 2);
   for (const auto& grp : at.groups) {
     attntc::Params p;
     p.b0 = grp.b0;
@@ -527,6 +531,8 @@ void launch_attn_tc(Exec& ex, const AttnTc& at) {
     p.Hk = sh.Hk;
     for (int i = 0; i < attntc::kMaxReq; ++i) p.S[i] = i < grp.nreq ? grp.S[i] : 0;
     p.q_tiles = q_tiles;
+    p.items = items;
+    p.pairs = pairs;
     p.splits = at.splits;
     p.rows_total = rows_total;
     p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
@@ -534,7 +540,7 @@ void launch_attn_tc(Exec& ex, const AttnTc& at) {
     p.part_o = at.part_o;
     p.part_ml = at.part_ml;
     p.err = ex.err;
-    dim3 grid(q_tiles * sh.Hq, grp.nreq, at.splits);
+    dim3 grid(sh.Hk * pairs, grp.nreq, at.splits);
     launch_pdl(attntc::attn_tc_kernel, grid, dim3(attntc::kThreads), attntc::kSmemBytes, ex.stream,
                *reinterpret_cast<const attntc::Maps*>(grp.maps), p);
     ex.launches++;

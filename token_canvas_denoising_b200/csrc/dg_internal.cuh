@@ -139,10 +139,17 @@ void launch_lmhead_simple(Exec& ex, int dtype, const void* hs, const void* W, co
 
 // tcgen05 LM head (bf16): vocab partitions for M rows, tensor maps, launch
 int lmhead_tc_partitions(int M, int V, int sm_count);
+// With fp8, hs and lm_head are e4m3 codes ([M][d] and [V][d] bytes) and the
+// launch takes their power-of-two row scales sa [M] and sw [V] (sa == null:
+// bf16 operands).
 bool lmhead_tc_prepare(const void* hs, const void* lm_head, int M, int d, int V, CUtensorMap* tmA,
-                       CUtensorMap* tmB);
+                       CUtensorMap* tmB, bool fp8 = false);
 void launch_lmhead_tc(Exec& ex, const CUtensorMap& tmA, const CUtensorMap& tmB, LmPartials part,
-                      const float* invT, int M, int d, int V);
+                      const float* invT, int M, int d, int V, const float* sa = nullptr,
+                      const float* sw = nullptr);
+// Quantize rows of a bf16 matrix to e4m3 with the smallest power-of-two scale
+// per row that fits the row's largest magnitude: codes [M][d], scales [M].
+void launch_quantize_rows_e4m3(Exec& ex, const void* x, uint8_t* codes, float* scales, int M, int d);
 
 // tcgen05 projection GEMM (bf16): out_i = A W_i^T (+ R) for up to 3 output
 // segments sharing A; prepared once (tensor maps), launched many times.
@@ -179,7 +186,7 @@ struct AttnTc {
   int splits = 1;
   std::vector<Group> groups;
 };
-int attn_tc_splits(int B, int C, int Hq, const int* S, int sm_count);
+int attn_tc_splits(int B, int C, int Hq, int Hk, const int* S, int sm_count);
 bool attn_tc_prepare(AttnTc* at, const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
                      const int32_t* S, const void* const* pk, const void* const* pv, void* O, float* part_o,
                      float* part_ml, int splits);
@@ -189,6 +196,7 @@ void launch_attn_tc(Exec& ex, const AttnTc& at);
 // combine; all buffers in one workspace region of moe_workspace_bytes().
 struct MoeShape {
   int M, d, E, topk, nsh, I;
+  bool fp8 = false;  // e4m3 expert weights
 };
 struct MoeTc {
   MoeShape s{};
@@ -203,13 +211,21 @@ struct MoeTc {
   void* xg = nullptr;        // [R][d] bf16
   void* act = nullptr;       // [R][I] bf16
   float* y = nullptr;        // [R][d]
+  uint8_t* xg8 = nullptr;    // e4m3: quantized token rows [R][d] and their scales sx [R]
+  uint8_t* act8 = nullptr;   // e4m3: quantized intermediate [R][I] and its scales sa [R]
+  float* sx = nullptr;
+  float* sa = nullptr;
+  const float* w_scale[3] = {nullptr, nullptr, nullptr};  // e4m3: row scales of W_gate, W_up, W_down
   GemmTc router;
   alignas(64) unsigned char maps_gateup[3 * 128];
   alignas(64) unsigned char maps_down[3 * 128];
 };
 size_t moe_workspace_bytes(const MoeShape& s);
+// With s.fp8 the expert weights are e4m3 codes and w_scales their row scales
+// (W_gate, W_up, W_down; [E+nsh][rows] f32 each).
 bool moe_prepare(MoeTc* mt, const MoeShape& s, const void* hs, void* hs_out, const void* w_router,
-                 const void* w_gate, const void* w_up, const void* w_down, void* ws, int sm_count);
+                 const void* w_gate, const void* w_up, const void* w_down, void* ws, int sm_count,
+                 const float* const* w_scales = nullptr);
 void launch_moe(Exec& ex, const MoeTc& mt);
 
 // ---- canvas bookkeeping
@@ -260,16 +276,24 @@ struct dg_ctx {
   // activations, storage dtype
   void *X = nullptr, *Q = nullptr, *Kc = nullptr, *Vc = nullptr, *O = nullptr;
   void *Hs = nullptr, *Hs2 = nullptr;
+  uint8_t* hs8 = nullptr;      // e4m3 LM head: the quantized residual stream [M][d]
+  float* hs8_scale = nullptr;  // and its row scales [M]
   dg::PrefixDesc* d_prefix = nullptr;
 
   dg::LmPartials lm{};
   float* ent = nullptr;
   int32_t* am = nullptr;
 
-  // tensor maps (bf16 path)
+  // attention layers: per layer the projection GEMMs and the attention
+  // (bf16 path); the residual stream after layer l is xres[l + 1] (xres[0] =
+  // X, the embedding; xres[L] = Hs, the input of the MoE block / LM head)
+  int L = 1;
+  std::vector<void*> xres;
   CUtensorMap tm_lm_a, tm_lm_b;
-  dg::GemmTc g_qkv, g_wo;
-  dg::AttnTc attn;
+  std::vector<dg::GemmTc> g_qkv, g_wo;
+  std::vector<dg::AttnTc> attn;
+  float* attn_part_o = nullptr;   // split-KV partials, shared by the layers
+  float* attn_part_ml = nullptr;
   int attn_splits = 1;
   int attn_splits_cap = 1;  // split partial buffers in the workspace are sized for this many
   dg::MoeTc moe;
@@ -284,7 +308,8 @@ struct dg_ctx {
   dg_schedule graph_sched{};
   int graph_launches = 0;
   // timing event pairs per timed kernel (DG_KERNEL_LMHEAD, DG_KERNEL_ATTENTION)
-  std::vector<cudaEvent_t> ev_start[2], ev_stop[2];
+  // and around the device-side decode loop (DG_KERNEL_DECODE)
+  std::vector<cudaEvent_t> ev_start[3], ev_stop[3];
   cudaEvent_t cur_ev_start[2] = {nullptr, nullptr}, cur_ev_stop[2] = {nullptr, nullptr};  // set while capturing
   // dg_decode_block's graph: the step as the body of a conditional while node
   cudaGraphExec_t decode_graph = nullptr;

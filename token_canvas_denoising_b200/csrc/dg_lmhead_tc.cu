@@ -22,6 +22,13 @@
 //
 // Warp roles: warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer,
 // warps 2..9 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31 of half (w-2)/4).
+//
+// FP8 variant (the FP8 deployment of "DiffusionGemma深度拆解", 性能数据): the
+// rows' activations and the vocab weights are e4m3 codes with power-of-two
+// scales (one per row of Hs, one per vocab row); the MMAs are kind::f8f6f4
+// (K = 32 per instruction, twice the K per 128-byte row), and the epilogue
+// multiplies each accumulated logit by its row's and its column's scale
+// before the online entropy/argmax (the product is exact for powers of two).
 #include "dg_internal.cuh"
 #include "dg_sm100.cuh"
 #include "dg_tmap.cuh"
@@ -32,7 +39,7 @@ namespace lmtc {
 using namespace sm100;
 
 constexpr int kStages = 3;
-constexpr int kBK = 64;                        // bf16 per 128-byte row
+constexpr int kRowBytes = 128;                 // one K block: 64 bf16 or 128 e4m3 per row
 constexpr int kHalfBytes = 128 * 128;          // 128 rows x 128 B
 constexpr int kABytes = 2 * kHalfBytes;        // 32 KB
 constexpr int kGranule = 32;                   // vocab columns per work granule
@@ -46,6 +53,8 @@ constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barrie
 struct Params {
   int M, d, V;
   const float* invT;  // [M] or null
+  const float* sa;    // FP8: [M] row scales of the activations
+  const float* sw;    // FP8: [V] row scales of the vocab weights
   LmRec* rec;         // [M][gridDim.x]
   int* err;
 };
@@ -56,8 +65,10 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  constexpr int kBK = kFp8 ? kRowBytes : kRowBytes / 2;  // K elements per block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
@@ -159,7 +170,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       for (int t = 0; t < n_tiles && !*abort_flag; ++t) {
         const int gt = g0 + t * kMaxGran;
         const int ng = min(kMaxGran, g1 - gt);
-        const uint32_t idesc = idesc_bf16_f32(128, ng * kGranule);
+        const uint32_t idesc = kFp8 ? idesc_e4m3_f32(128, ng * kGranule) : idesc_bf16_f32(128, ng * kGranule);
         if (!mbar_wait(tempty, tph ^ 1u, p.err, abort_flag)) break;
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
@@ -171,10 +182,13 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           for (int h = 0; h < 2; ++h) {
             if (h < halves) {
 #pragma unroll
-              for (int k = 0; k < kBK / 16; ++k) {
+              for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
                 const uint64_t ad = umma_desc_sw128(a0 + h * kHalfBytes + k * 32, 16, 1024);
                 const uint64_t bd = umma_desc_sw128(b0 + k * 32, 16, 1024);
-                mma_bf16_ss(tmem + h * 256, ad, bd, idesc, (kb | k) != 0);
+                if constexpr (kFp8)
+                  mma_f8_ss(tmem + h * 256, ad, bd, idesc, (kb | k) != 0);
+                else
+                  mma_bf16_ss(tmem + h * 256, ad, bd, idesc, (kb | k) != 0);
               }
             }
           }
@@ -200,6 +214,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const bool has_row = half < halves && row < p.M;
     const float kLog2e = 1.4426950408889634f;
     const float it2 = (has_row && p.invT ? p.invT[row] : 1.f) * kLog2e;  // logit -> scaled base-2
+    const float sa = kFp8 && has_row ? p.sa[row] : 1.f;
     float m2 = -INFINITY, z0 = 0.f, z1 = 0.f, s0 = 0.f, s1 = 0.f, best = -INFINITY;
     int idx = 0x7fffffff;
     uint32_t tph = 0;
@@ -214,11 +229,14 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           uint32_t r[32];
           tmem_ld32_sync(tbase + c0, r);
           const int vbase = gt * kGranule + c0;
+          // FP8: this lane's column scale, handed to the other lanes below
+          const float swl = kFp8 ? __ldg(p.sw + vbase + lane) * sa : 1.f;
           float l[32];
           float bm = -INFINITY;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(r[i]);
+            float x = __uint_as_float(r[i]);
+            if constexpr (kFp8) x *= __shfl_sync(0xffffffffu, swl, i);
             if (x > best) { best = x; idx = vbase + i; }
             l[i] = x * it2;
             bm = fmaxf(bm, l[i]);
@@ -282,33 +300,42 @@ int lmhead_tc_partitions(int M, int V, int sm_count) {
 }
 
 bool lmhead_tc_prepare(const void* hs, const void* lm_head, int M, int d, int V, CUtensorMap* tmA,
-                       CUtensorMap* tmB) {
+                       CUtensorMap* tmB, bool fp8) {
   // kernel attributes are set here, on the host path that precedes any launch
   // (and never inside a stream capture)
-  if (cudaFuncSetAttribute(lmtc::lmhead_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           lmtc::kSmemBytes) != cudaSuccess) {
+  if (cudaFuncSetAttribute(fp8 ? lmtc::lmhead_tc_kernel<true> : lmtc::lmhead_tc_kernel<false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, lmtc::kSmemBytes) != cudaSuccess) {
     set_last_error("cudaFuncSetAttribute(lmhead_tc_kernel) failed");
     return false;
   }
+  // one box = 128 bytes of K (64 bf16 or 128 e4m3) x 256 rows
+  const uint64_t es = fp8 ? 1 : 2;
   const uint64_t dA[2] = {(uint64_t)d, (uint64_t)M};
-  const uint64_t sA[1] = {(uint64_t)d * 2};
-  const uint32_t bA[2] = {64, 256};
+  const uint64_t sA[1] = {(uint64_t)d * es};
+  const uint32_t bA[2] = {(uint32_t)(lmtc::kRowBytes / es), 256};
   const uint64_t dB[2] = {(uint64_t)d, (uint64_t)V};
-  const uint32_t bB[2] = {64, (uint32_t)(lmtc::kMaxGran * lmtc::kGranule)};
+  const uint32_t bB[2] = {(uint32_t)(lmtc::kRowBytes / es), (uint32_t)(lmtc::kMaxGran * lmtc::kGranule)};
+  if (fp8)
+    return encode_tmap_u8(tmA, hs, 2, dA, sA, bA, true) && encode_tmap_u8(tmB, lm_head, 2, dB, sA, bB, true);
   return encode_tmap_bf16(tmA, hs, 2, dA, sA, bA, true) && encode_tmap_bf16(tmB, lm_head, 2, dB, sA, bB, true);
 }
 
 void launch_lmhead_tc(Exec& ex, const CUtensorMap& tmA, const CUtensorMap& tmB, LmPartials part,
-                      const float* invT, int M, int d, int V) {
+                      const float* invT, int M, int d, int V, const float* sa, const float* sw) {
   lmtc::Params p;
   p.M = M;
   p.d = d;
   p.V = V;
   p.invT = invT;
+  p.sa = sa;
+  p.sw = sw;
   p.rec = part.rec;
   p.err = ex.err;
   dim3 grid(part.P, ceil_div(M, 256));
-  launch_pdl(lmtc::lmhead_tc_kernel, grid, dim3(lmtc::kThreads), lmtc::kSmemBytes, ex.stream, tmA, tmB, p);
+  if (sa)
+    launch_pdl(lmtc::lmhead_tc_kernel<true>, grid, dim3(lmtc::kThreads), lmtc::kSmemBytes, ex.stream, tmA, tmB, p);
+  else
+    launch_pdl(lmtc::lmhead_tc_kernel<false>, grid, dim3(lmtc::kThreads), lmtc::kSmemBytes, ex.stream, tmA, tmB, p);
   ex.launches++;
 }
 

@@ -14,6 +14,14 @@
 //   combine  Hs2 = bf16(Hs + sum_k g_k y_k + sum_shared y_shared), summed in
 //            slot order so the result does not depend on scheduling
 //
+// With e4m3 expert weights (the FP8 deployment of "DiffusionGemma深度拆解",
+// 性能数据) the weights are e4m3 codes with power-of-two scales per output row,
+// the gathered token rows and the GeGLU intermediate are quantized per row
+// (dg_fp8.cu) ahead of the gate/up and the down GEMMs, the MMAs are
+// kind::f8f6f4 over 128-byte K blocks (a K tail past moe_inter is zero-filled
+// by the tensor map), and the epilogues multiply by the weight row's and the
+// token row's scales.
+//
 // The expert GEMMs put the weights on the 128-row MMA side (M = 128 rows of
 // W) and an expert's tokens (a few dozen) on the N side, so a CTA streams one
 // 128-row weight tile of one expert through a TMA ring while its tokens' rows
@@ -205,6 +213,9 @@ struct FfnParams {
   int rows;            // weight rows: I (gate/up) or d (down)
   __nv_bfloat16* act;  // gate/up output [R][I]
   float* y;            // down output [R][d]
+  const float* sw0;    // e4m3: row scales of W_gate (gate/up) or W_down (down), [E+nsh][rows]
+  const float* sw1;    // e4m3: row scales of W_up (gate/up)
+  const float* sx;     // e4m3: token row scales, [R]
   int* err;
 };
 
@@ -214,8 +225,9 @@ __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.f + er
 // K block by the same B (the expert's token rows). MODE 0: a 128-row tile of
 // W_gate and of W_up, GeGLU epilogue to act. MODE 1: a 256-row tile of W_down
 // (one box) as two 128-row halves, f32 y.
-template <int MODE>
+template <int MODE, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_constant__ FfnMaps maps, FfnParams p) {
+  constexpr int kBK = FP8 ? 128 : 64;  // K elements per 128-byte block
   griddep_launch();
   griddep_wait();  // the routing offsets and the B rows come from the previous kernels
   const int e = blockIdx.y, rt = blockIdx.x;
@@ -224,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
   if (n <= 0) return;  // expert without tokens (uniform over the CTA)
   const int N = (n + 15) & ~15;
   const int nbox = (n + kBox - 1) / kBox;
-  const int nk = p.K / 64;
+  const int nk = (p.K + kBK - 1) / kBK;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -268,13 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
         uint8_t* st = smem + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], bytes);
         if (MODE == 0) {
-          tma_load_3d(st, &maps.a0, &full[s], kb * 64, rt * 128, e, polW);
-          tma_load_3d(st + kATile, &maps.a1, &full[s], kb * 64, rt * 128, e, polW);
+          tma_load_3d(st, &maps.a0, &full[s], kb * kBK, rt * 128, e, polW);
+          tma_load_3d(st + kATile, &maps.a1, &full[s], kb * kBK, rt * 128, e, polW);
         } else {
-          tma_load_3d(st, &maps.a0, &full[s], kb * 64, rt * 256, e, polW);  // 256 rows = both halves
+          tma_load_3d(st, &maps.a0, &full[s], kb * kBK, rt * 256, e, polW);  // 256 rows = both halves
         }
         for (int bx = 0; bx < nbox; ++bx)
-          tma_load_2d(st + 2 * kATile + bx * kBox * 128, &maps.b, &full[s], kb * 64, r0 + bx * kBox, polX);
+          tma_load_2d(st + 2 * kATile + bx * kBox * 128, &maps.b, &full[s], kb * kBK, r0 + bx * kBox, polX);
         issued[s] = true;
         iph[s] = ph;
         if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -285,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, N);
+      const uint32_t idesc = FP8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N);
       int s = 0;
       uint32_t ph = 0;
       for (int kb = 0; kb < nk; ++kb) {
@@ -294,10 +306,15 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
         const uint32_t a0 = smem_u32(smem + s * kStageBytes);
         const uint32_t b0 = a0 + 2 * kATile;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
           const uint64_t bd = umma_desc_sw128(b0 + k * 32, 16, 1024);
-          mma_bf16_ss(tmem, umma_desc_sw128(a0 + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
-          mma_bf16_ss(tmem + 256, umma_desc_sw128(a0 + kATile + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
+          if constexpr (FP8) {
+            mma_f8_ss(tmem, umma_desc_sw128(a0 + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
+            mma_f8_ss(tmem + 256, umma_desc_sw128(a0 + kATile + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
+          } else {
+            mma_bf16_ss(tmem, umma_desc_sw128(a0 + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
+            mma_bf16_ss(tmem + 256, umma_desc_sw128(a0 + kATile + k * 32, 16, 1024), bd, idesc, (kb | k) != 0);
+          }
         }
         mma_commit(&empty[s]);
         if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -311,6 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const bool ok = mbar_wait_warp(tfull, 0, p.err, abort_flag);
     tc_fence_after();
+    // e4m3: this thread's weight-row scales (both halves of a down tile)
+    float ws0 = 1.f, ws1 = 1.f;
+    if (FP8 && ok) {
+      const size_t base = (size_t)e * p.rows;
+      if (row < p.rows) ws0 = p.sw0[base + row];
+      if (MODE == 0 && row < p.rows) ws1 = p.sw1[base + row];
+      if (MODE == 1 && row + 128 < p.rows) ws1 = p.sw0[base + row + 128];
+    }
     if (ok) {
       for (int c = 0; c < (n + 31) / 32; ++c) {
         uint32_t g[32];
@@ -323,7 +348,13 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
             for (int j = 0; j < 32; ++j) {
               const int tok = c * 32 + j;
               if (tok < n) {
-                const float a = gelu_erf(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
+                if constexpr (FP8) {
+                  const float sx = __ldg(p.sx + r0 + tok);
+                  gv *= ws0 * sx;
+                  uv *= ws1 * sx;
+                }
+                const float a = gelu_erf(gv) * uv;
                 p.act[(size_t)(r0 + tok) * p.rows + row] = __float2bfloat16_rn(a);
               }
             }
@@ -334,8 +365,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_ffn_kernel(const __grid_const
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int tok = c * 32 + j;
-            if (tok < n && row < p.rows) p.y[(size_t)(r0 + tok) * p.rows + row] = __uint_as_float(g[j]);
-            if (tok < n && row + 128 < p.rows) p.y[(size_t)(r0 + tok) * p.rows + row + 128] = __uint_as_float(g1[j]);
+            const float sx = (FP8 && tok < n) ? __ldg(p.sx + r0 + tok) : 1.f;
+            if (tok < n && row < p.rows) p.y[(size_t)(r0 + tok) * p.rows + row] = __uint_as_float(g[j]) * (ws0 * sx);
+            if (tok < n && row + 128 < p.rows)
+              p.y[(size_t)(r0 + tok) * p.rows + row + 128] = __uint_as_float(g1[j]) * (ws1 * sx);
           }
         }
       }
@@ -396,18 +429,19 @@ size_t moe_workspace_bytes(const MoeShape& s) {
   return al(sizeof(float) * s.M * s.E) + al(sizeof(float) * s.M * s.topk) + al(sizeof(int) * s.M * s.topk) +
          al(sizeof(int) * s.M * (s.topk + s.nsh)) +
          al(sizeof(int) * (s.E + s.nsh + 1)) + al(sizeof(int) * R) + al(2 * R * s.d) + al(2 * R * s.I) +
-         al(4 * R * s.d) + 8 * 256;
+         al(4 * R * s.d) + (s.fp8 ? al(R * s.d) + al(R * s.I) + 2 * al(4 * R) : 0) + 12 * 256;
 }
 
 bool moe_prepare(MoeTc* mt, const MoeShape& s, const void* hs, void* hs_out, const void* w_router, const void* w_gate,
-                 const void* w_up, const void* w_down, void* ws, int sm_count) {
+                 const void* w_up, const void* w_down, void* ws, int sm_count, const float* const* w_scales) {
   if (s.E > moe::kMaxE || s.topk > moe::kMaxTopK || s.M * s.topk > moe::kMaxPairs || s.nsh < 0 || s.nsh > 2 ||
-      s.I % 64 != 0 || s.d % 64 != 0) {
+      s.I % 64 != 0 || s.d % 64 != 0 || (s.fp8 && s.d % 128 != 0)) {
     set_last_error("MoE: unsupported sizes (E <= 256, top_k <= 8, M*top_k <= 8192, n_shared <= 2, "
-                   "moe_inter and d_model multiples of 64)");
+                   "moe_inter and d_model multiples of 64, d_model a multiple of 128 with e4m3 experts)");
     return false;
   }
-  for (auto f : {(const void*)moe::moe_ffn_kernel<0>, (const void*)moe::moe_ffn_kernel<1>})
+  for (auto f : {(const void*)moe::moe_ffn_kernel<0, false>, (const void*)moe::moe_ffn_kernel<1, false>,
+                 (const void*)moe::moe_ffn_kernel<0, true>, (const void*)moe::moe_ffn_kernel<1, true>})
     if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, moe::kSmemBytes) != cudaSuccess) {
       set_last_error("cudaFuncSetAttribute(moe_ffn_kernel) failed");
       return false;
@@ -431,6 +465,13 @@ bool moe_prepare(MoeTc* mt, const MoeShape& s, const void* hs, void* hs_out, con
   mt->xg = take(2 * R * s.d);
   mt->act = take(2 * R * s.I);
   mt->y = reinterpret_cast<float*>(take(4 * R * s.d));
+  if (s.fp8) {
+    mt->xg8 = reinterpret_cast<uint8_t*>(take(R * s.d));
+    mt->act8 = reinterpret_cast<uint8_t*>(take(R * s.I));
+    mt->sx = reinterpret_cast<float*>(take(4 * R));
+    mt->sa = reinterpret_cast<float*>(take(4 * R));
+    for (int i = 0; i < 3; ++i) mt->w_scale[i] = w_scales[i];
+  }
   // router: f32 logits, one K split (no partial buffer needed)
   const void* wr[1] = {w_router};
   void* lo[1] = {mt->logits};
@@ -452,6 +493,20 @@ bool moe_prepare(MoeTc* mt, const MoeShape& s, const void* hs, void* hs_out, con
   const uint64_t dx[2] = {(uint64_t)s.d, R}, sx[1] = {(uint64_t)s.d * 2};
   const uint64_t da[2] = {(uint64_t)s.I, R}, sa[1] = {(uint64_t)s.I * 2};
   const uint32_t bb[2] = {64, (uint32_t)moe::kBox};
+  if (s.fp8) {  // e4m3 codes: one byte per element, 128-byte K boxes
+    const uint64_t sgu8[2] = {(uint64_t)s.d, (uint64_t)s.I * s.d};
+    const uint64_t sdn8[2] = {(uint64_t)s.I, (uint64_t)s.d * s.I};
+    const uint32_t bw8[3] = {128, 128, 1};
+    const uint32_t bw_dn8[3] = {128, 256, 1};
+    const uint64_t sx8[1] = {(uint64_t)s.d}, sa8[1] = {(uint64_t)s.I};
+    const uint32_t bb8[2] = {128, (uint32_t)moe::kBox};
+    return encode_tmap_u8(&gu->a0, w_gate, 3, dgu, sgu8, bw8, true) &&
+           encode_tmap_u8(&gu->a1, w_up, 3, dgu, sgu8, bw8, true) &&
+           encode_tmap_u8(&gu->b, mt->xg8, 2, dx, sx8, bb8, true) &&
+           encode_tmap_u8(&dn->a0, w_down, 3, ddn, sdn8, bw_dn8, true) &&
+           encode_tmap_u8(&dn->a1, w_down, 3, ddn, sdn8, bw_dn8, true) &&
+           encode_tmap_u8(&dn->b, mt->act8, 2, da, sa8, bb8, true);
+  }
   if (!encode_tmap_bf16(&gu->a0, w_gate, 3, dgu, sgu, bw, true) || !encode_tmap_bf16(&gu->a1, w_up, 3, dgu, sgu, bw, true) ||
       !encode_tmap_bf16(&gu->b, mt->xg, 2, dx, sx, bb, true) || !encode_tmap_bf16(&dn->a0, w_down, 3, ddn, sdn, bw_dn, true) ||
       !encode_tmap_bf16(&dn->a1, w_down, 3, ddn, sdn, bw_dn, true) || !encode_tmap_bf16(&dn->b, mt->act, 2, da, sa, bb, true))
@@ -485,12 +540,28 @@ void launch_moe(Exec& ex, const MoeTc& mt) {
   fp.y = mt.y;
   fp.K = s.d;
   fp.rows = s.I;
-  launch_pdl(moe::moe_ffn_kernel<0>, dim3(ceil_div(s.I, 128), s.E + s.nsh), dim3(moe::kThreads), moe::kSmemBytes,
-             ex.stream, *reinterpret_cast<const moe::FfnMaps*>(mt.maps_gateup), fp);
+  fp.sw0 = mt.w_scale[0];
+  fp.sw1 = mt.w_scale[1];
+  fp.sx = mt.sx;
+  const dim3 g_gu(ceil_div(s.I, 128), s.E + s.nsh), g_dn(ceil_div(s.d, 256), s.E + s.nsh);
+  const moe::FfnMaps& m_gu = *reinterpret_cast<const moe::FfnMaps*>(mt.maps_gateup);
+  const moe::FfnMaps& m_dn = *reinterpret_cast<const moe::FfnMaps*>(mt.maps_down);
+  if (s.fp8) {
+    launch_quantize_rows_e4m3(ex, mt.xg, mt.xg8, mt.sx, R, s.d);
+    launch_pdl(moe::moe_ffn_kernel<0, true>, g_gu, dim3(moe::kThreads), moe::kSmemBytes, ex.stream, m_gu, fp);
+    launch_quantize_rows_e4m3(ex, mt.act, mt.act8, mt.sa, R, s.I);
+  } else {
+    launch_pdl(moe::moe_ffn_kernel<0, false>, g_gu, dim3(moe::kThreads), moe::kSmemBytes, ex.stream, m_gu, fp);
+  }
   fp.K = s.I;
   fp.rows = s.d;
-  launch_pdl(moe::moe_ffn_kernel<1>, dim3(ceil_div(s.d, 256), s.E + s.nsh), dim3(moe::kThreads), moe::kSmemBytes,
-             ex.stream, *reinterpret_cast<const moe::FfnMaps*>(mt.maps_down), fp);
+  fp.sw0 = mt.w_scale[2];
+  fp.sw1 = nullptr;
+  fp.sx = mt.sa;
+  if (s.fp8)
+    launch_pdl(moe::moe_ffn_kernel<1, true>, g_dn, dim3(moe::kThreads), moe::kSmemBytes, ex.stream, m_dn, fp);
+  else
+    launch_pdl(moe::moe_ffn_kernel<1, false>, g_dn, dim3(moe::kThreads), moe::kSmemBytes, ex.stream, m_dn, fp);
   launch_pdl(moe::moe_combine_kernel, dim3(s.M), dim3(256), 0, ex.stream, static_cast<const __nv_bfloat16*>(mt.hs),
              (const float*)mt.y, (const int*)mt.pos, (const float*)mt.gate, static_cast<__nv_bfloat16*>(mt.hs_out), s.d,
              s.topk, s.nsh);

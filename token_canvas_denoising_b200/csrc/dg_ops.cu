@@ -76,6 +76,7 @@ dg_status dg_lmhead_entropy(int32_t dtype, const void* hs, const void* lm_head, 
   if (dg_status est = make_exec(stream, &ex)) return est;
   dg::LmPartials part;
   part.P = dtype == DG_BF16 ? dg::lmhead_tc_partitions(M, V, ex.sm_count) : std::max(1, std::min(128, V / 1024));
+  part.rec = nullptr;
   dg_status st = cuda_status(cudaMallocAsync((void**)&part.rec, sizeof(dg::LmRec) * (size_t)M * part.P, ex.stream),
                              "cudaMallocAsync");
   if (st != DG_OK) return st;
@@ -93,6 +94,47 @@ dg_status dg_lmhead_entropy(int32_t dtype, const void* hs, const void* lm_head, 
   st = cuda_status(cudaGetLastError(), "launch");
   cudaFreeAsync(part.rec, ex.stream);
   return st;
+}
+
+dg_status dg_lmhead_entropy_e4m3(const void* hs, const void* lm_head, const float* lm_scale, const float* inv_temp,
+                                 int32_t M, int32_t d, int32_t V, float* ent, int32_t* argmax, void* stream) {
+  OP_ARG(hs && lm_head && lm_scale && ent && argmax, "NULL buffer");
+  OP_ARG(M >= 1 && d >= 1 && V >= 2, "sizes");
+  OP_ARG(al16(hs) && al16(lm_head), "hs / lm_head must be 16-byte aligned");
+  OP_UNSUP(d % 128 == 0 && V % 256 == 0, "the e4m3 LM head needs d % 128 == 0 and V % 256 == 0");
+  dg::Exec ex;
+  if (dg_status est = make_exec(stream, &ex)) return est;
+  dg::LmPartials part;
+  part.P = dg::lmhead_tc_partitions(M, V, ex.sm_count);
+  uint8_t* q = nullptr;
+  float* sa = nullptr;
+  dg_status st = cuda_status(cudaMallocAsync((void**)&part.rec, sizeof(dg::LmRec) * (size_t)M * part.P, ex.stream),
+                             "cudaMallocAsync");
+  if (st == DG_OK) st = cuda_status(cudaMallocAsync((void**)&q, (size_t)M * d, ex.stream), "cudaMallocAsync");
+  if (st == DG_OK) st = cuda_status(cudaMallocAsync((void**)&sa, sizeof(float) * M, ex.stream), "cudaMallocAsync");
+  CUtensorMap a, b;
+  if (st == DG_OK && !dg::lmhead_tc_prepare(q, lm_head, M, d, V, &a, &b, true)) st = DG_ERR_CUDA;
+  if (st == DG_OK) {
+    dg::launch_quantize_rows_e4m3(ex, hs, q, sa, M, d);
+    dg::launch_lmhead_tc(ex, a, b, part, inv_temp, M, d, V, sa, lm_scale);
+    dg::launch_merge_select(ex, part, ent, argmax, nullptr, nullptr, nullptr, 1, M, V);
+    st = cuda_status(cudaGetLastError(), "launch");
+  }
+  if (sa) cudaFreeAsync(sa, ex.stream);
+  if (q) cudaFreeAsync(q, ex.stream);
+  if (part.rec) cudaFreeAsync(part.rec, ex.stream);
+  return st;
+}
+
+dg_status dg_quantize_rows_e4m3(const void* x, uint8_t* codes, float* scales, int32_t M, int32_t d, void* stream) {
+  OP_ARG(x && codes && scales, "NULL buffer");
+  OP_ARG(M >= 1 && d >= 1, "sizes");
+  OP_ARG(al16(x) && (reinterpret_cast<uintptr_t>(codes) & 7u) == 0, "x must be 16-byte and codes 8-byte aligned");
+  OP_UNSUP(d % 8 == 0, "d % 8 != 0");
+  dg::Exec ex;
+  if (dg_status est = make_exec(stream, &ex)) return est;
+  dg::launch_quantize_rows_e4m3(ex, x, codes, scales, M, d);
+  return cuda_status(cudaGetLastError(), "launch");
 }
 
 dg_status dg_attention(int32_t dtype, const void* q, const void* kc, const void* vc, int32_t B, int32_t C,
@@ -114,7 +156,7 @@ dg_status dg_attention(int32_t dtype, const void* q, const void* kc, const void*
   if (dtype == DG_BF16) {
     OP_ARG(al16(q) && al16(kc) && al16(vc) && al16(o), "buffers must be 16-byte aligned");
     dg::AttnShape sh{B, C, Hq, Hk, h};
-    const int splits = dg::attn_tc_splits(B, C, Hq, prefix_len, ex.sm_count);
+    const int splits = dg::attn_tc_splits(B, C, Hq, Hk, prefix_len, ex.sm_count);
     float* part = nullptr;
     const size_t rows = (size_t)B * C * Hq;
     if (splits > 1) {

@@ -67,20 +67,49 @@ __device__ __forceinline__ uint32_t float_order(float f) {
 }
 
 constexpr int kMaxRecPerLane = 8;  // partials preloaded per lane (P <= 256 in one pass)
+constexpr int kMaxSelect = 1024;   // positions per canvas the selection sorts (one per thread)
 
-// Grid (ceil(C/8), B), 256 threads. Phase 1: one warp per canvas row folds the
-// row's P partials (lane j takes partials j, j+32, ..., all loaded before the
-// fold; then a fixed xor butterfly), giving ent = ln Z - S/Z and the argmax.
-// Phase 2 runs in the last block of each canvas to arrive: each unfrozen
-// position counts the unfrozen positions with a smaller (entropy, position)
-// key; the k with rank < k freeze to their argmax; stop test; re-noise. The
-// last canvas to finish sets the all-done flag.
-__global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
+// Ascending bitonic sort of one 64-bit key per thread across the block
+// (blockDim.x a power of two, at most kMaxSelect): compare-exchange stages
+// with partner distances below 32 run inside a warp through shuffles, the
+// others through shared memory. Afterwards thread t holds the t-th smallest.
+__device__ __forceinline__ unsigned long long block_bitonic_sort(unsigned long long key,
+                                                                 unsigned long long* s_x) {
+  const int t = threadIdx.x, n = blockDim.x;
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      unsigned long long other;
+      if (stride >= 32) {
+        s_x[t] = key;
+        __syncthreads();
+        other = s_x[t ^ stride];
+        __syncthreads();
+      } else {
+        other = __shfl_xor_sync(0xffffffffu, key, stride);
+      }
+      const bool up = (t & size) == 0;      // this run is sorted ascending
+      const bool lower = (t & stride) == 0;  // lower element of the pair
+      key = (lower == up) ? (other < key ? other : key) : (other > key ? other : key);
+    }
+  }
+  return key;
+}
+
+// Grid (ceil(C / (blockDim/32)), B), blockDim the power of two >= C between
+// 256 and 1024. Phase 1: one warp per canvas row folds the row's P partials
+// (lane j takes partials j, j+32, ..., all loaded before the fold; then a
+// fixed xor butterfly), giving ent = ln Z - S/Z and the argmax. Phase 2 runs
+// in the last block of each canvas to arrive: the unfrozen positions' keys
+// (entropy, position) are sorted across the block (frozen and padding slots
+// sort last); the first k freeze to their argmax; stop test; re-noise. The
+// last canvas to finish sets the all-done flag (and ends a device-side decode
+// loop).
+__global__ void __launch_bounds__(kMaxSelect) merge_select_kernel(SelectArgs a) {
   griddep_launch();
   griddep_wait();
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p_row = blockIdx.x * 8 + warp;
+  const int p_row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (p_row < a.C) {
     const int r = b * a.C + p_row;
     const LmRec* rec = a.part.rec + (size_t)r * a.part.P;
@@ -125,8 +154,9 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
   if (!s_last) return;
   __threadfence();
 
-  __shared__ __align__(16) unsigned long long s_key[256];
-  __shared__ float s_min[8];
+  __shared__ unsigned long long s_x[kMaxSelect];
+  __shared__ uint8_t s_freeze[kMaxSelect];
+  __shared__ float s_min[kMaxSelect / 32];
   const int p = threadIdx.x;
   const bool valid = p < a.C;
   const int r = b * a.C + p;
@@ -140,22 +170,16 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
     // key = (entropy, position); frozen and padding slots sort after every unfrozen one
     const unsigned long long key =
         unf ? (((unsigned long long)float_order(e) << 32) | (unsigned)p) : ~0ull;
-    s_key[p] = key;
     const int U = __syncthreads_count(unf);
     const int t = a.step[b];
     const int left = a.max_steps - t;
     const int k = (left <= 1) ? U : (U + left - 1) / left;
-    bool F = false;
-    if (unf) {
-      int rank = 0;
-      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(s_key);
-#pragma unroll 8
-      for (int q = 0; q < 128; ++q) {
-        const ulonglong2 kq = k2[q];
-        rank += (kq.x < key) + (kq.y < key);
-      }
-      F = rank < k;
-    }
+    const unsigned long long sorted = block_bitonic_sort(key, s_x);
+    s_freeze[p] = 0;
+    __syncthreads();
+    if (p < k) s_freeze[(unsigned)(sorted & 0xffffffffu)] = 1;  // k <= U: an unfrozen position
+    __syncthreads();
+    const bool F = unf && s_freeze[p];
     const int amv = valid ? __ldcg(&a.am[r]) : 0;
     if (F) {
       a.tok[r] = amv;
@@ -169,8 +193,7 @@ __global__ void __launch_bounds__(256) merge_select_kernel(SelectArgs a) {
     if (lane == 0) s_min[warp] = mr;
     const int R = __syncthreads_count(rest);
     float min_rest = s_min[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) min_rest = fminf(min_rest, s_min[w]);
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) min_rest = fminf(min_rest, s_min[w]);
     const bool stop = (R == 0) || (a.adaptive && min_rest < a.stop_entropy);
     if (stop) {
       if (rest) a.tok[r] = amv;
@@ -235,8 +258,12 @@ void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uin
       a.loop_cap = loop->cap;
     }
   }
-  dim3 grid(ceil_div(C, 8), B);
-  launch_pdl(merge_select_kernel, grid, dim3(256), 0, ex.stream, a);
+  // one thread per position in the selection: the power of two >= C, at
+  // least 256 (phase 1 then folds blockDim/32 rows per block)
+  int threads = 256;
+  while (threads < C && threads < kMaxSelect) threads <<= 1;
+  dim3 grid(ceil_div(C, threads / 32), B);
+  launch_pdl(merge_select_kernel, grid, dim3(threads), 0, ex.stream, a);
   ex.launches++;
 }
 

@@ -20,8 +20,23 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   return fn;
 }
 
+static bool encode_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       bool swizzle128);
+
 bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                       const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128) {
+  return encode_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box, swizzle128);
+}
+
+bool encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128) {
+  return encode_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides_bytes, box, swizzle128);
+}
+
+static bool encode_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank,
+                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                       bool swizzle128) {
   auto fn = get_encoder();
   if (!fn) {
     set_last_error("cuTensorMapEncodeTiled is not available");
@@ -36,7 +51,7 @@ bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64
     es[i] = 1;
     if (i + 1 < rank) gs[i] = strides_bytes[i];
   }
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = fn(map, type, rank, const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -13,6 +13,11 @@ namespace dg {
 bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                       const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
 
+// The same for an 8-bit element type (e4m3 codes), encoded as unsigned bytes:
+// dims[0] and box[0] count bytes.
+bool encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+
 // The calling thread's current CUDA context (driver handle), or false when
 // none can be read. Used to key per-context caches of device addresses.
 bool current_context(void** ctx);

@@ -14,7 +14,8 @@ Workloads follow the five synthetic configurations of the method's hot path
   longctx    B4 C256 S32768  d2816 Hq16/Hk8 h128 V262144  bf16  T=48, prefix scale U[0.5, 2] per (request, head)
   moe        vocab262k + MoE 128 experts + 1 shared, top-8, GeGLU intermediate 704
   *_fp8      vocab262k / longctx with the LM head stored as e4m3 codes and
-             power-of-two row scales (the FP8 deployment the pages report)
+             power-of-two row scales (the FP8 deployment the pages report);
+             moe_fp8 also stores the expert weights that way
 
 Weights are N(0, std) with std = 1/sqrt(fan_in), fan_in being the contraction
 dimension of the matrix; the embedding table uses std 1 (a one-hot lookup reads
@@ -57,6 +58,7 @@ class Config:
     stop_entropy: float = 0.05
     lm_fp8: bool = False           # LM head stored as e4m3 codes with power-of-two row scales
     n_layers: int = 0              # 0: one layer, unstacked arrays; L >= 1: L layers stacked [L][...]
+    moe_fp8: bool = False          # expert weights stored as e4m3 codes with power-of-two row scales
 
     @property
     def M(self):
@@ -81,6 +83,7 @@ CONFIGS = {
 }
 CONFIGS["vocab262k_fp8"] = replace(CONFIGS["vocab262k"], name="vocab262k_fp8", lm_fp8=True)
 CONFIGS["longctx_fp8"] = replace(CONFIGS["longctx"], name="longctx_fp8", lm_fp8=True)
+CONFIGS["moe_fp8"] = replace(CONFIGS["moe"], name="moe_fp8", lm_fp8=True, moe_fp8=True)
 CONFIG_ORDER = ["tiny", "canvas256", "vocab262k", "longctx", "moe"]
 
 
@@ -195,6 +198,13 @@ def make_workload(cfg, weight_overrides=None):
                 ("w_down", (c.d, c.moe_inter), 1.0 / math.sqrt(c.moe_inter), 3000)):
             if name in ov:
                 w[name] = ov.pop(name)
+                continue
+            if c.moe_fp8:  # the same draws, stored as e4m3 codes with row scales
+                codes = np.empty((ne,) + shape, dtype=np.uint8)
+                sc = np.empty((ne, shape[0]), dtype=np.float32)
+                for e in range(ne):
+                    codes[e], sc[e] = e4m3_rows(normal(c.weight_seed, base + e, shape, std, "f32"))
+                w[name], w[name + "_scale"] = codes, sc
                 continue
             arr = np.empty((ne,) + shape, dtype=np.uint16 if dt == "bf16" else np.float32)
             for e in range(ne):

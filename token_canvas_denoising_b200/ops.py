@@ -37,6 +37,21 @@ def lmhead_entropy(hs, lm_head, inv_temp=None):
     return ent, am
 
 
+def lmhead_entropy_e4m3(hs, lm_codes, lm_scale, inv_temp=None):
+    """The LM head with e4m3 weights: hs bf16 [M][d] (quantized per row inside),
+    lm_codes uint8 [V][d] e4m3 codes, lm_scale f32 [V] row scales (powers of
+    two). Returns (entropy f32 [M], argmax int32 [M])."""
+    lib = L.load()
+    M, d = hs.shape
+    V = lm_codes.shape[0]
+    ent = torch.empty(M, dtype=torch.float32, device=hs.device)
+    am = torch.empty(M, dtype=torch.int32, device=hs.device)
+    st = lib.dg_lmhead_entropy_e4m3(_p(hs), _p(lm_codes), _p(lm_scale), _p(inv_temp), M, d, V, _p(ent), _p(am),
+                                    _stream())
+    L.check(st, "dg_lmhead_entropy_e4m3")
+    return ent, am
+
+
 def lmhead_entropy_noalloc(hs, lm_head, inv_temp=None, ent=None, argmax=None):
     """Like lmhead_entropy, but the library makes no device allocation: its
     temporary partial results live in a fixed device array inside the library.

@@ -1,7 +1,7 @@
 """Run the denoise step on a named synthetic workload, for profilers.
 
     python -m token_canvas_denoising_b200.profile_ops [--workload canvas256] [--steps 6]
-        [--op step|lmhead|attention|linear]
+        [--op step|lmhead|lmhead_e4m3|attention|linear]
 
 'step' runs CUDA-graph denoise steps through the C ABI (every kernel of the
 path); the other ops run the single-operation entry points on the workload's
@@ -23,7 +23,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="canvas256")
     ap.add_argument("--steps", type=int, default=6)
-    ap.add_argument("--op", default="step", choices=["step", "lmhead", "attention", "linear"])
+    ap.add_argument("--op", default="step", choices=["step", "lmhead", "lmhead_e4m3", "attention", "linear"])
     a = ap.parse_args()
     cfg = fx.CONFIGS[a.workload]
     torch.cuda.set_device(0)
@@ -48,6 +48,11 @@ def main():
             hs = to_device(fx.normal(7, 1, (M, d), 1.0, "bf16"), "bf16", "cuda")
             w = to_device(fx.normal(7, 2, (V, d), 1.0 / math.sqrt(d), "bf16"), "bf16", "cuda")
             run = lambda: ops.lmhead_entropy(hs, w)
+        elif a.op == "lmhead_e4m3":
+            hs = to_device(fx.normal(7, 1, (M, d), 1.0, "bf16"), "bf16", "cuda")
+            codes, scales = fx.e4m3_rows(fx.normal(7, 2, (V, d), 1.0 / math.sqrt(d), "f32"))
+            w, sw = torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()
+            run = lambda: ops.lmhead_entropy_e4m3(hs, w, sw)
         elif a.op == "linear":
             N = (cfg.Hq + 2 * cfg.Hk) * cfg.h
             x = to_device(fx.normal(7, 1, (M, d), 1.0, "bf16"), "bf16", "cuda")

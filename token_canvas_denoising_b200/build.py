@@ -2,12 +2,17 @@
 
     python -m token_canvas_denoising_b200.build [--force] [-v]
 
-Each .cu under csrc/ is compiled to an object (rebuilt when it or a header is
-newer than the object) and the objects are linked into a shared library next
-to this file. The CUDA runtime is linked statically.
+Each .cu under csrc/ is compiled to an object and the objects are linked into
+a shared library next to this file. An object is rebuilt unless the hash
+recorded beside it equals the hash of its source, every header and the
+compiler command (file times are not trusted: a copied tree can carry
+objects newer than their sources); the library is relinked whenever an object
+was rebuilt or the recorded hash of the object set differs. The CUDA runtime
+is linked statically.
 """
 import argparse
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -40,15 +45,35 @@ def headers():
     return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+def _digest(paths, extra):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(os.path.relpath(p, ROOT).encode() + b"\0" + f.read())
+    h.update(" ".join(os.path.relpath(x, ROOT) if os.path.isabs(x) else x for x in extra).encode())
+    return h.hexdigest()
+
+
+def _recorded(path):
+    try:
+        with open(path) as f:
+            return f.read().strip()
+    except OSError:
+        return None
+
+
 def build(force=False, verbose=False, jobs=None):
     os.makedirs(BUILD, exist_ok=True)
-    hdr_mtime = max((os.path.getmtime(h) for h in headers()), default=0)
-    objs, cmds = [], []
+    hdrs = headers()
+    objs, cmds, stamps = [], [], []
     for src in sources():
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
-        if (force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr_mtime)):
-            cmds.append([nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj])
+        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+        digest = _digest([src] + hdrs, cmd[1:])
+        if force or not os.path.exists(obj) or _recorded(obj + ".sha256") != digest:
+            cmds.append(cmd)
+            stamps.append((obj + ".sha256", digest))
     procs = []
     for cmd in cmds:
         if verbose:
@@ -65,13 +90,19 @@ def build(force=False, verbose=False, jobs=None):
     if failed:
         msg = "\n".join(f"--- {src}\n{txt}" for src, txt in failed)
         raise RuntimeError("nvcc failed:\n" + msg)
-    if cmds or not os.path.exists(LIB) or force:
-        link = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-cudart", "static"]
+    for path, digest in stamps:
+        with open(path, "w") as f:
+            f.write(digest + "\n")
+    link = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-cudart", "static"]
+    lib_digest = _digest(objs, link[1:])
+    if cmds or force or not os.path.exists(LIB) or _recorded(LIB + ".sha256") != lib_digest:
         if verbose:
             print(" ".join(link), flush=True)
         r = subprocess.run(link, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n" + r.stdout.decode(errors="replace"))
+        with open(LIB + ".sha256", "w") as f:
+            f.write(lib_digest + "\n")
     return LIB
 
 

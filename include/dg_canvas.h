@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define DG_ABI_VERSION 1
+#define DG_ABI_VERSION 2
 
 typedef enum dg_status {
   DG_OK = 0,

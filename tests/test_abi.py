@@ -46,7 +46,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings_and_version(lib):
     from token_canvas_denoising_b200 import _lib
-    assert lib.dg_abi_version() == 1
+    assert lib.dg_abi_version() == 2
     for s in range(7):
         assert lib.dg_status_string(s)
     assert lib.dg_status_string(_lib.DG_ERR_OOM) == b"out of device memory"
@@ -151,3 +151,59 @@ def test_product_binding_has_no_fallback(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         _lib.load()
+
+
+@pytest.mark.parametrize("field,value", [("n_layers", -1), ("n_layers", 65), ("lm_head_format", 7),
+                                         ("expert_format", 3)])
+def test_init_rejects_bad_model_fields(lib, field, value):
+    m = _model()
+    setattr(m, field, value)
+    ctx = C.c_void_p()
+    plen = (C.c_int32 * 1)(0)
+    seeds = (C.c_uint64 * 1)(0)
+    st = lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None, None,
+                            C.cast(seeds, C.c_void_p), None)
+    assert st == 1 and not ctx.value
+
+
+def test_init_rejects_e4m3_without_scales_or_with_f32(lib):
+    from token_canvas_denoising_b200 import _lib
+    ctx = C.c_void_p()
+    plen = (C.c_int32 * 1)(0)
+    seeds = (C.c_uint64 * 1)(0)
+    m = _model(**_BF16)
+    m.lm_head_format = _lib.DG_LM_E4M3  # no lm_head_scale
+    assert lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None, None,
+                              C.cast(seeds, C.c_void_p), None) == 1
+    m.lm_head_scale = 4096
+    m.d_model = 192  # not a multiple of 128
+    assert lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None, None,
+                              C.cast(seeds, C.c_void_p), None) == 2
+    m = _model()  # f32 storage
+    m.lm_head_format, m.lm_head_scale = _lib.DG_LM_E4M3, 4096
+    assert lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None, None,
+                              C.cast(seeds, C.c_void_p), None) == 2
+    m = _model(**dict(_BF16, **_MOE))
+    m.expert_format = _lib.DG_LM_E4M3  # no expert scales
+    assert lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None, None,
+                              C.cast(seeds, C.c_void_p), None) == 1
+    assert not ctx.value
+
+
+def test_init_rejects_moe_with_a_layer_stack(lib):
+    m = _model(**dict(_BF16, **_MOE))
+    m.n_layers = 2
+    ctx = C.c_void_p()
+    plen = (C.c_int32 * 1)(0)
+    seeds = (C.c_uint64 * 1)(0)
+    st = lib.dg_canvas_init(C.byref(ctx), C.byref(m), 1, 16, C.cast(plen, C.c_void_p), None, None, None,
+                            C.cast(seeds, C.c_void_p), None)
+    assert st == 2 and b"single-layer" in lib.dg_last_error()
+
+
+def test_op_entry_points_reject_bad_arguments(lib):
+    assert lib.dg_lmhead_entropy_e4m3(None, None, None, None, 4, 128, 256, None, None, None) == 1
+    buf = C.c_void_p(4096)
+    assert lib.dg_lmhead_entropy_e4m3(buf, buf, buf, None, 4, 96, 256, buf, buf, None) == 2  # d % 128
+    assert lib.dg_quantize_rows_e4m3(None, None, None, 4, 128, None) == 1
+    assert lib.dg_quantize_rows_e4m3(buf, buf, buf, 4, 12, None) == 2  # d % 8

@@ -270,6 +270,10 @@ dg_status dg_canvas_set_kernel_timing(dg_ctx *ctx, int32_t kernel, int32_t n, vo
 /* dg_canvas_set_kernel_timing(ctx, DG_KERNEL_LMHEAD, n, starts, stops). */
 dg_status dg_canvas_set_timing_events(dg_ctx *ctx, int32_t n, void *const *starts, void *const *stops);
 
+/* Steps run by the device-side loop of the most recent dg_decode_block (0
+ * before the first), into host *steps_out. Synchronous. */
+dg_status dg_canvas_loop_steps(dg_ctx *ctx, int32_t *steps_out);
+
 /* Wait for the context's stream and report device-side errors (synchronous). */
 dg_status dg_canvas_sync(dg_ctx *ctx);
 

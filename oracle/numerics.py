@@ -66,9 +66,8 @@ def widen(w, dtype):
 E4M3_MAX = 448.0
 
 
-def e4m3_to_f64(codes):
-    """e4m3 byte codes -> float64 (exact)."""
-    b = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+def _e4m3_value(b):
+    """The value of e4m3 byte codes b (int64 array), from the format's definition."""
     sign = np.where((b & 0x80) != 0, -1.0, 1.0)
     e = (b >> 3) & 0xF
     m = (b & 7).astype(np.float64)
@@ -77,7 +76,16 @@ def e4m3_to_f64(codes):
     return sign * mag
 
 
-_E4M3_NONNEG = e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))  # codes 0..126, increasing
+_E4M3_TABLE = _e4m3_value(np.arange(256, dtype=np.int64))  # the 256 codes' values
+
+
+def e4m3_to_f64(codes):
+    """e4m3 byte codes -> float64 (exact; a lookup in the table of the 256
+    codes' values)."""
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+_E4M3_NONNEG = _E4M3_TABLE[:0x7F]  # codes 0..126, increasing
 
 
 def round_to_e4m3(x):

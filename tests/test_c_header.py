@@ -31,7 +31,8 @@ def _program():
              "                     (fn)dg_canvas_reset_fixed, (fn)dg_canvas_block_kv, (fn)dg_canvas_set_prefix,",
              "                     (fn)dg_lmhead_entropy, (fn)dg_lmhead_entropy_e4m3,",
              "                     (fn)dg_quantize_rows_e4m3, (fn)dg_lmhead_entropy_noalloc, (fn)dg_attention,",
-             "                     (fn)dg_linear, (fn)dg_ops_check, (fn)dg_selftest_wait_timeout};",
+             "                     (fn)dg_linear, (fn)dg_ops_check, (fn)dg_selftest_wait_timeout,",
+             "                     (fn)dg_canvas_loop_steps};",
              "  (void)f;"]
     for s, fields in STRUCTS.items():
         lines.append(f'  printf("{s} size %zu\\n", sizeof({s}));')

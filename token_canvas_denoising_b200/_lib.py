@@ -57,6 +57,7 @@ SIGNATURES = {
     "dg_canvas_get_state": (C.c_int, [C.c_void_p, C.POINTER(dg_state)]),
     "dg_canvas_set_state": (C.c_int, [C.c_void_p, C.POINTER(dg_state)]),
     "dg_canvas_sync": (C.c_int, [C.c_void_p]),
+    "dg_canvas_loop_steps": (C.c_int, [C.c_void_p, C.c_void_p]),
     "dg_canvas_reset": (C.c_int, [C.c_void_p, C.c_void_p]),
     "dg_canvas_reset_fixed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "dg_canvas_block_kv": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),

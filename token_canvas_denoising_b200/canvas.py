@@ -194,6 +194,12 @@ class DenoiseCanvas:
         st = self._lib.dg_canvas_set_kernel_timing(self._ctx, k, n, C.cast(a, C.c_void_p), C.cast(b, C.c_void_p))
         L.check(st, "dg_canvas_set_kernel_timing")
 
+    def loop_steps(self):
+        """Steps run by the device-side loop of the most recent decode()."""
+        n = C.c_int32(0)
+        L.check(self._lib.dg_canvas_loop_steps(self._ctx, C.byref(n)), "dg_canvas_loop_steps")
+        return int(n.value)
+
     def sync(self):
         L.check(self._lib.dg_canvas_sync(self._ctx), "dg_canvas_sync")
 

@@ -581,6 +581,7 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   cudaStream_t sm = c->ex.stream;
   if (cudaMemcpyAsync(c->cs.seed, seeds, batch * sizeof(uint64_t), cudaMemcpyHostToDevice, sm) != cudaSuccess ||
       cudaMemsetAsync(c->cs.counters, 0, (batch + 1) * sizeof(uint32_t), sm) != cudaSuccess ||
+      cudaMemsetAsync(c->cs.loop_iter, 0, sizeof(int32_t), sm) != cudaSuccess ||
       cudaMemsetAsync(c->err, 0, sizeof(int32_t), sm) != cudaSuccess) {
     set_last_error("initial copies failed");
     return fail(DG_ERR_CUDA);
@@ -766,6 +767,13 @@ dg_status dg_canvas_set_kernel_timing(dg_ctx* ctx, int32_t kernel, int32_t n, vo
 
 dg_status dg_canvas_set_timing_events(dg_ctx* ctx, int32_t n, void* const* starts, void* const* stops) {
   return dg_canvas_set_kernel_timing(ctx, DG_KERNEL_LMHEAD, n, starts, stops);
+}
+
+dg_status dg_canvas_loop_steps(dg_ctx* ctx, int32_t* steps_out) {
+  DG_ARG(ctx != nullptr && steps_out != nullptr, "NULL argument");
+  DG_CUDA_RET(cudaMemcpyAsync(steps_out, ctx->cs.loop_iter, sizeof(int32_t), cudaMemcpyDeviceToHost, ctx->ex.stream));
+  DG_CUDA_RET(cudaStreamSynchronize(ctx->ex.stream));
+  return DG_OK;
 }
 
 dg_status dg_canvas_sync(dg_ctx* ctx) {

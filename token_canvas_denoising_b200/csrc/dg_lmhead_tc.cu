@@ -229,14 +229,15 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           uint32_t r[32];
           tmem_ld32_sync(tbase + c0, r);
           const int vbase = gt * kGranule + c0;
-          // FP8: this lane's column scale, handed to the other lanes below
-          const float swl = kFp8 ? __ldg(p.sw + vbase + lane) * sa : 1.f;
+          // FP8: lane i loads the scale of column vbase + i and hands it to
+          // the other lanes; each thread applies it with its own row's scale
+          const float swl = kFp8 ? __ldg(p.sw + vbase + lane) : 1.f;
           float l[32];
           float bm = -INFINITY;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             float x = __uint_as_float(r[i]);
-            if constexpr (kFp8) x *= __shfl_sync(0xffffffffu, swl, i);
+            if constexpr (kFp8) x *= __shfl_sync(0xffffffffu, swl, i) * sa;
             if (x > best) { best = x; idx = vbase + i; }
             l[i] = x * it2;
             bm = fmaxf(bm, l[i]);

@@ -85,9 +85,10 @@ def test_lmhead_prescribed_logits():
 
 
 @pytest.mark.parametrize("M", [256, 1024])
-def test_lmhead_full_vocab_sampled_rows(M):
-    """V = 262,144, d = 2816 (the vocab262k / longctx shapes); 12 sampled rows
-    against the oracle, every row's entropy within [0, ln V]."""
+def test_lmhead_full_vocab_every_row(M):
+    """V = 262,144, d = 2816 (the vocab262k / longctx shapes): every row
+    against the oracle (entropy within 1e-3 nats, argmax equal outside
+    near-ties) and within [0, ln V]."""
     from token_canvas_denoising_b200 import ops
     d, V = 2816, 262144
     hs = fx.normal(41, 1, (M, d), 1.0, "bf16")
@@ -96,7 +97,9 @@ def test_lmhead_full_vocab_sampled_rows(M):
     ent, am = ops.lmhead_entropy(_dev(hs), _dev(w), torch.from_numpy(invT).cuda())
     ent, am = ent.cpu().numpy(), am.cpu().numpy()
     assert np.all(ent >= -1e-4) and np.all(ent <= math.log(V) + 1e-3)
-    rows = np.random.default_rng(M).choice(M, 12, replace=False)
-    rows[0], rows[-1] = 0, M - 1
-    ent_o, am_o, gap_o = _oracle(hs, w, invT, rows)
-    _check(ent[rows], am[rows], ent_o, am_o, gap_o)
+    wf = on.bf16_bits_to_f64(w)  # widened once for the row blocks below
+    for r0 in range(0, M, 256):
+        rows = np.arange(r0, min(M, r0 + 256))
+        logits = om.lm_head_logits({"dtype": "bf16", "lm_head": wf}, on.bf16_bits_to_f64(hs[rows]))
+        ent_o, am_o, gap_o = om.entropy_argmax(logits, invT[rows].astype(np.float64))
+        _check(ent[rows], am[rows], ent_o, am_o, gap_o)

@@ -104,6 +104,9 @@ __device__ __forceinline__ unsigned long long block_bitonic_sort(unsigned long l
 // sort last); the first k freeze to their argmax; stop test; re-noise. The
 // last canvas to finish sets the all-done flag (and ends a device-side decode
 // loop).
+// kLoop: the step is the body of a device-side decode loop (a.cond set); only
+// that instantiation contains the call that sets the loop's condition.
+template <bool kLoop>
 __global__ void __launch_bounds__(kMaxSelect) merge_select_kernel(SelectArgs a) {
   griddep_launch();
   griddep_wait();
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(kMaxSelect) merge_select_kernel(SelectArgs a) 
       for (int i = 0; i < a.B; ++i) all &= (__ldcg(&a.done[i]) != 0) ? 1 : 0;
       *a.all_done = all;
       a.counters[a.B] = 0;
-      if (a.cond) {  // the step is the body of a device-side decode loop
+      if constexpr (kLoop) {  // the step is the body of a device-side decode loop
         const int it = *a.loop_iter + 1;
         *a.loop_iter = it;
         if (!all && it >= a.loop_cap) set_error(a.err, kDevLoopCap);
@@ -263,7 +266,10 @@ void launch_merge_select(Exec& ex, LmPartials part, float* ent, int32_t* am, uin
   int threads = 256;
   while (threads < C && threads < kMaxSelect) threads <<= 1;
   dim3 grid(ceil_div(C, threads / 32), B);
-  launch_pdl(merge_select_kernel, grid, dim3(threads), 0, ex.stream, a);
+  if (a.cond)
+    launch_pdl(merge_select_kernel<true>, grid, dim3(threads), 0, ex.stream, a);
+  else
+    launch_pdl(merge_select_kernel<false>, grid, dim3(threads), 0, ex.stream, a);
   ex.launches++;
 }
 

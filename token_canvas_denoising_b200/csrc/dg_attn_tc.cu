@@ -31,8 +31,7 @@
 //              P_x (bf16 pairs) over the first 64 columns of S_x. While one
 //              slot's warps exponentiate, the tensor core runs the other
 //              slot's MMAs, so the MUFU and the tensor pipe stay busy
-//              together; half of the exponentials run on the FMA pipe
-//              (exp2_poly). The running maximum is raised only when the tile's
+//              together. The running maximum is raised only when the tile's
 //              maximum exceeds it by more than 8 (a factor 256), and then O_x
 //              and the running sum are rescaled in place; the decision is per
 //              warp, since the TMEM accesses are warp-collective.
@@ -96,26 +95,6 @@ struct Params {
   float* part_ml;    // [splits][rows_total][2]
   int* err;
 };
-
-// 2^x on the FMA and integer pipes, for x >= -125 (smaller x, including the
-// -inf of masked keys, clamp to 2^-125, which a bf16 P and the row sum treat
-// as 0): a Cody-Waite split x = j + f, with j = x rounded to the nearest
-// integer (read from the low mantissa bits of x + 1.5 * 2^23, so no conversion
-// instruction) and f = x - j in [-1/2, 1/2]; 2^f from a degree-3 polynomial
-// fitted for this kernel to 2^f on [-1/2, 1/2] in relative error (largest
-// relative error 7.6e-5, far below the 2^-9 half-ulp of the bf16 P it feeds);
-// 2^j by adding j to the exponent field. The softmax sends half of its
-// exponentials here and half to ex2.approx on the MUFU, which would otherwise
-// bound the kernel (one pair of query tiles needs 32K exponentials per key
-// tile; the MUFU retires 8 per clock per SM).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;  // 1.5 * 2^23
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05517052486538887f, f, 0.24260830879211426f), f, 0.693260908126831f), f,
-                       0.9999282360076904f);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
 
 __device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
   // K-major 128-row operand with 128 columns of K split into two 64-wide atoms
@@ -361,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const float p0 = ex2_approx(fmaf(v[2 * c], p.scale_log2, neg_m));
-        const float p1 = exp2_poly(fmaf(v[2 * c + 1], p.scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(v[2 * c + 1], p.scale_log2, neg_m));
         ls[(2 * c) & 7] += p0;
         ls[(2 * c + 1) & 7] += p1;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
@@ -479,15 +458,12 @@ int attn_ctas_per_request(int C, int Hq, int Hk) {
 }  // namespace attntc
 
 // ---------------------------------------------------------------- host side
-// KV splits: enough CTAs to fill the SMs, but at least 3 key tiles per split
-// (a CTA's set-up -- TMEM, barriers, two Q tiles, the first K/V fetches -- and
-// its share of the merge cost about one key tile each).
 int attn_tc_splits(int B, int C, int Hq, int Hk, const int* S, int sm_count) {
   const int q_tiles = ceil_div(C, 128);
   int min_tiles = 1 << 30;
   for (int b = 0; b < B; ++b) min_tiles = std::min(min_tiles, ceil_div(S[b], 128) + q_tiles);
   int splits = sm_count / std::max(1, B * attntc::attn_ctas_per_request(C, Hq, Hk));
-  splits = std::max(1, std::min(splits, std::min(min_tiles / 3, 16)));
+  splits = std::max(1, std::min(splits, std::min(min_tiles, 16)));
   return splits;
 }
 

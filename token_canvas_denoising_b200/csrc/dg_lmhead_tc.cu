@@ -65,26 +65,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA and integer pipes for x <= 0 (x < -125 clamps to about
-// 2^-125, which adds at most V 2^-125 to a sum of at least 1): a Cody-Waite
-// split x = j + f, j = x rounded to the nearest integer (read from the low
-// mantissa bits of x + 1.5 * 2^23), f = x - j in [-1/2, 1/2]; 2^f from a
-// degree-4 polynomial fitted for this kernel to 2^f on [-1/2, 1/2] in
-// relative error (largest relative error 2.7e-6: the entropy ln Z - S/Z then
-// moves by at most 2 * 2.7e-6 * ln V < 7e-5 nats); 2^j by adding j to the
-// exponent field. A third of the epilogue's exponentials run here: the MUFU
-// retires 8 per clock per SM, and with this split its time and the epilogue's
-// issue slots balance.
-__device__ __forceinline__ float exp2_poly4(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;  // 1.5 * 2^23
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(fmaf(0.009569993242621422f, f, 0.055917542427778244f), f, 0.240247443318367f), f,
-                            0.6931218504905701f),
-                       f, 0.9999992847442627f);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
-
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
@@ -276,8 +256,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const float d0 = l[i] - m2, d1 = l[i + 1] - m2;
-            const float e0 = (i % 6 == 4) ? exp2_poly4(d0) : ex2(d0);  // 5 of 32 on the FMA pipe
-            const float e1 = (i % 6 == 2) ? exp2_poly4(d1) : ex2(d1);  // and 5 more: about a third
+            const float e0 = ex2(d0), e1 = ex2(d1);
             z0 += e0;
             z1 += e1;
             s0 = fmaf(d0, e0, s0);

@@ -174,8 +174,9 @@ typedef struct dg_ctx dg_ctx;
  *   prefix_k/v  host arrays of B device pointers, each [S_b][n_kv_heads][head_dim]
  *               in the storage dtype ([L][S_b][...] with n_layers = L > 1; NULL
  *               allowed when S_b = 0).
- *   inv_temp    device [B*C] f32 per-position inverse temperature applied to the
- *               logits before the entropy, or NULL for 1.
+ *   inv_temp    device [B*C] f32 per-position inverse temperature (>= 0) applied
+ *               to the logits before the entropy, or NULL for 1; a negative
+ *               value gives an undefined entropy.
  *   seeds       host [B] Philox seeds; canvas b position p starts at
  *               draw(seeds[b], step 0, p, b).
  *   cuda_stream cudaStream_t to queue all work on (NULL = default stream).

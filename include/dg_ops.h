@@ -29,7 +29,8 @@ extern "C" {
  *   x[r][v] = hs[r] . lm_head[v]          (f32 accumulate)
  *   ent[r]  = H(softmax(x[r] * inv_temp[r])) in nats
  *   argmax[r] = argmax_v x[r][v] (lowest v on ties)
- * hs [M][d], lm_head [V][d] (dtype); inv_temp [M] f32 or NULL (= 1);
+ * hs [M][d], lm_head [V][d] (dtype); inv_temp [M] f32 >= 0 or NULL (= 1; a
+ * negative inverse temperature gives an undefined entropy);
  * ent [M] f32, argmax [M] int32 (outputs). The logits are never stored.
  * bf16 needs d % 64 == 0 and V % 256 == 0; f32 any d % 8 == 0. */
 dg_status dg_lmhead_entropy(int32_t dtype, const void *hs, const void *lm_head, const float *inv_temp,

@@ -51,24 +51,25 @@ def test_lmhead_random(M, d, V):
     _check(ent.cpu().numpy(), am.cpu().numpy(), ent_o, am_o, gap_o)
 
 
-def test_lmhead_prescribed_logits():
-    """Hs rows are unit vectors e_0, so logit[r][v] = W[v][0] exactly: one-hot
-    rows give entropy 0, constant rows give ln V, and equal maxima in two
-    different CTAs' vocab ranges resolve to the lower id."""
+@pytest.mark.parametrize("M", [4, 200])
+def test_lmhead_prescribed_logits(M):
+    """Hs rows are unit vectors e_0, so logit[r][v] = W[v][0] exactly: three
+    equal maxima give entropy ln 3 and resolve to the lowest id (12300 and
+    12345 fall in one 256-column tile, in different column halves of a CTA
+    pair's epilogue; 40000 in another partition's range); constant rows give
+    ln V; one-hot rows give entropy 0. M = 4 runs on single CTAs, M = 200 on
+    CTA pairs (rows 128.. in the odd CTA)."""
     from token_canvas_denoising_b200 import ops
-    M, d, V = 4, 64, 65536
+    d, V = 64, 65536
     hs = np.zeros((M, d), np.float32)
     hs[:, 0] = 1.0
-    w = np.zeros((V, d), np.float32)
-    logits = np.full((M, V), -1000.0, np.float32)
-    # row 0: one-hot at 12345; row 1: all equal (set below by a separate W column)
     hs_bits = fx.f32_to_bf16_bits(hs)
+    w = np.zeros((V, d), np.float32)
     w[:, 0] = -1000.0
-    w[12345, 0] = 0.0
-    w[40000, 0] = 0.0   # a tie with 12345 in another CTA's range for row 0
+    w[[40000, 12345, 12300], 0] = 0.0
     ent, am = ops.lmhead_entropy(_dev(hs_bits), _dev(fx.f32_to_bf16_bits(w)))
     ent, am = ent.cpu().numpy(), am.cpu().numpy()
-    assert abs(ent[0] - math.log(2.0)) < 1e-5 and am[0] == 12345
+    assert np.all(np.abs(ent - math.log(3.0)) < 1e-5) and np.all(am == 12300)
     # constant logits: ln V
     w2 = np.zeros((V, d), np.float32)
     w2[:, 0] = 0.25

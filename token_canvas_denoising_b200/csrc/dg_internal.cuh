@@ -128,6 +128,28 @@ inline void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// launch_pdl for kernels whose CTAs run in pairs (thread-block clusters of 2
+// along x, for tcgen05 .cta_group::2): grid.x must be even.
+template <typename... KArgs, typename... Args>
+inline void launch_pdl_pairs(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = t_pdl_off ? 1 : 2;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---- embed / linear / attention / LM head (dtype-dispatched)
 void launch_embed(Exec& ex, int dtype, const void* E, const int32_t* tok, void* X, int M, int d, int V);
 void launch_linear_simple(Exec& ex, int dtype, const void* A, const void* W, const void* R, void* out,

@@ -446,11 +446,13 @@ def bench_b200(args, rank, world, local_rank):
     # when the timed kernels ran under it too, or ran a second or more
     capped = "sw_power_cap" in (ck or {}).get("reasons", [])
     peak_kind = "sustained" if (region2_s >= SUSTAINED_AFTER_S or capped) else "burst"
-    lm = kernel_roofline("lmhead", "lmhead_tc_kernel<" + ("e4m3" if cfg.lm_fp8 else "bf16")
+    # more than 128 rows run on CTA pairs (lmhead_tc_pair_kernel)
+    lm_kernel = "lmhead_tc_pair_kernel" if cfg.B * cfg.C > 128 else "lmhead_tc_kernel"
+    lm = kernel_roofline("lmhead", lm_kernel + "<" + ("e4m3" if cfg.lm_fp8 else "bf16")
                          + "> (LM head + entropy/argmax)", fb["flops_lm"], fb["bytes_lm"],
-                         float(np.mean(dur["lmhead"])), peaks, peak_kind, traffic_of("lmhead_tc_kernel", cfg.name),
+                         float(np.mean(dur["lmhead"])), peaks, peak_kind, traffic_of(lm_kernel, cfg.name),
                          fp8=cfg.lm_fp8)
-    at = kernel_roofline("attention", "attn_tc_kernel (+ attn_merge_kernel when split)", fb["flops_attn"],
+    at = kernel_roofline("attention", "attn_tc_kernel (+ attn_merge_kernel for units shared by CTAs)", fb["flops_attn"],
                          fb["bytes_attn"], float(np.mean(dur["attention"])), peaks, peak_kind,
                          traffic_of("attn_tc_kernel", cfg.name))
 

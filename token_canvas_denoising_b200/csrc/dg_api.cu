@@ -102,10 +102,10 @@ void layout_workspace(dg_ctx* c, void* base, size_t* total) {
       c->g_wo[l].part = po;
     }
   }
-  if (c->m.dtype == DG_BF16 && c->attn_splits > 1) {
+  if (c->m.dtype == DG_BF16 && c->attn_slots > 1) {
     const size_t rows = M * (size_t)c->m.n_q_heads;
-    c->attn_part_o = w.take<float>((size_t)c->attn_splits * rows * 128);
-    c->attn_part_ml = w.take<float>((size_t)c->attn_splits * rows * 2);
+    c->attn_part_o = w.take<float>((size_t)c->attn_slots * rows * 128);
+    c->attn_part_ml = w.take<float>((size_t)c->attn_slots * rows * 2);
   }
   *total = w.off + 256;
 }
@@ -216,7 +216,7 @@ dg_status prepare_layer_attention(dg_ctx* c) {
     if (c->m.dtype == DG_BF16) {
       dg::AttnShape sh{c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads, c->m.head_dim};
       if (!dg::attn_tc_prepare(&c->attn[l], sh, c->Q, c->Kc, c->Vc, c->S.data(), pk.data(), pv.data(), c->O,
-                               c->attn_part_o, c->attn_part_ml, c->attn_splits))
+                               c->attn_part_o, c->attn_part_ml, c->attn_slots, c->ex.sm_count))
         return DG_ERR_CUDA;
     }
   }
@@ -528,8 +528,8 @@ dg_status dg_canvas_init(dg_ctx** out, const dg_model_desc* model, int32_t batch
   }
   if (model->dtype == DG_BF16) {
     c->lm.P = dg::lmhead_tc_partitions(c->M, model->vocab, c->ex.sm_count);
-    c->attn_splits = dg::attn_tc_splits(batch, canvas_len, model->n_q_heads, model->n_kv_heads, c->S.data(), c->ex.sm_count);
-    c->attn_splits_cap = c->attn_splits;
+    c->attn_slots = dg::attn_tc_slots(batch, canvas_len, model->n_q_heads, model->n_kv_heads, c->S.data(),
+                                      c->ex.sm_count);
     // tile / split choice only (buffers are bound after the workspace exists)
     const int qd = model->n_q_heads * model->head_dim, kd = model->n_kv_heads * model->head_dim;
     const void* wqkv[3] = {model->wq, model->wk, model->wv};
@@ -680,9 +680,8 @@ dg_status dg_canvas_set_prefix(dg_ctx* c, const int32_t* prefix_len, const void*
     c->pv[b] = prefix_len[b] ? prefix_v[b] : nullptr;
     c->max_S = std::max(c->max_S, (int)prefix_len[b]);
   }
-  if (c->m.dtype == DG_BF16)  // the split partial buffers were sized at init: never exceed that split count
-    c->attn_splits = std::min(c->attn_splits_cap, dg::attn_tc_splits(c->B, c->C, c->m.n_q_heads, c->m.n_kv_heads,
-                                                                    c->S.data(), c->ex.sm_count));
+  // the attention's partial buffers were sized at init: its schedule for the
+  // new lengths shares no unit among more CTAs than they hold
   dg_status st = prepare_layer_attention(c);
   if (st != DG_OK) return st;
   DG_CUDA_RET(cudaStreamSynchronize(c->ex.stream));

@@ -196,22 +196,33 @@ void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual);
 // tcgen05 attention (bf16, head_dim 128): tensor maps per group of up to 8
 // requests, split-KV partial buffers.
 struct AttnTc {
+  // stream-K schedule of one launch: the units' T key tiles over G CTAs, at
+  // most `parts` CTAs per unit (the partial slots it needs)
+  struct Sched {
+    int G = 1, T = 0, Tp = 0, parts = 1;
+    int nt[8] = {0}, reqoff[8] = {0};
+  };
   struct Group {
     alignas(64) unsigned char maps[19 * 128];
     int b0 = 0, nreq = 0;
     int S[8] = {0};
+    Sched sched;
   };
   AttnShape sh{};
   void* O = nullptr;
   float* part_o = nullptr;
   float* part_ml = nullptr;
-  int splits = 1;
   std::vector<Group> groups;
 };
-int attn_tc_splits(int B, int C, int Hq, int Hk, const int* S, int sm_count);
+// Partial slots (parts per row) the attention needs for these prefix lengths
+// on sm_count SMs; 1 = none.
+int attn_tc_slots(int B, int C, int Hq, int Hk, const int* S, int sm_count);
+// Tensor maps and schedules; the schedules share no unit among more than
+// `slots` CTAs (the partial buffers hold [slots][B*C*Hq] rows; with part_o
+// NULL every unit runs in one CTA).
 bool attn_tc_prepare(AttnTc* at, const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
                      const int32_t* S, const void* const* pk, const void* const* pv, void* O, float* part_o,
-                     float* part_ml, int splits);
+                     float* part_ml, int slots, int sm_count);
 void launch_attn_tc(Exec& ex, const AttnTc& at);
 
 // MoE FFN (bf16): router GEMM, routing, gather, expert gate/up and down GEMMs,
@@ -314,10 +325,9 @@ struct dg_ctx {
   CUtensorMap tm_lm_a, tm_lm_b;
   std::vector<dg::GemmTc> g_qkv, g_wo;
   std::vector<dg::AttnTc> attn;
-  float* attn_part_o = nullptr;   // split-KV partials, shared by the layers
+  float* attn_part_o = nullptr;   // attention partials (units shared by CTAs), shared by the layers
   float* attn_part_ml = nullptr;
-  int attn_splits = 1;
-  int attn_splits_cap = 1;  // split partial buffers in the workspace are sized for this many
+  int attn_slots = 1;             // partial slots per row the workspace holds
   dg::MoeTc moe;
   void* moe_ws = nullptr;
 

@@ -460,7 +460,10 @@ lmhead_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       const uint64_t polA = policy_evict_last();
-      const uint64_t polB = policy_evict_first();
+      // vocab rows: streamed once when one 256-row block reads them; with
+      // several blocks, the blocks' pairs read each row at slightly different
+      // times and the row should stay in L2 until the last of them
+      const uint64_t polB = gridDim.y > 1 ? policy_evict_normal() : policy_evict_first();
       const uint32_t full_even = mapa_shared(full, 0);
       const uint32_t tx = 2 * kPairStageBytes;  // both CTAs' boxes (rows past M or V are zero-filled, counted)
       int s = 0;

@@ -156,18 +156,18 @@ dg_status dg_attention(int32_t dtype, const void* q, const void* kc, const void*
   if (dtype == DG_BF16) {
     OP_ARG(al16(q) && al16(kc) && al16(vc) && al16(o), "buffers must be 16-byte aligned");
     dg::AttnShape sh{B, C, Hq, Hk, h};
-    const int splits = dg::attn_tc_splits(B, C, Hq, Hk, prefix_len, ex.sm_count);
+    const int slots = dg::attn_tc_slots(B, C, Hq, Hk, prefix_len, ex.sm_count);
     float* part = nullptr;
     const size_t rows = (size_t)B * C * Hq;
-    if (splits > 1) {
-      dg_status st = cuda_status(cudaMallocAsync((void**)&part, splits * rows * 130 * sizeof(float), ex.stream),
+    if (slots > 1) {
+      dg_status st = cuda_status(cudaMallocAsync((void**)&part, slots * rows * 130 * sizeof(float), ex.stream),
                                  "cudaMallocAsync");
       if (st != DG_OK) return st;
     }
     dg::AttnTc at;
     dg_status st = DG_OK;
     if (!dg::attn_tc_prepare(&at, sh, q, kc, vc, prefix_len, prefix_k, prefix_v, o, part,
-                             part ? part + splits * rows * 128 : nullptr, splits))
+                             part ? part + slots * rows * 128 : nullptr, slots, ex.sm_count))
       st = DG_ERR_CUDA;
     else {
       dg::launch_attn_tc(ex, at);

@@ -163,18 +163,24 @@ __global__ void __launch_bounds__(kMaxSelect) merge_select_kernel(SelectArgs a) 
   const int p = threadIdx.x;
   const bool valid = p < a.C;
   const int r = b * a.C + p;
+  // this block runs alone on the step's critical path: every load it needs
+  // is issued here together, and the re-noise draw (which depends only on
+  // the seed, the step and the position) is computed before the sort
   const bool canvas_done = __ldcg(&a.done[b]) != 0;
+  float e = valid ? __ldcg(&a.ent[r]) : INFINITY;
+  const bool unf = valid && __ldcg(&a.frozen[r]) == 0;
+  const int amv = valid ? __ldcg(&a.am[r]) : 0;
+  const int t = __ldcg(&a.step[b]);
+  const uint64_t seed = __ldcg(&a.seed[b]);
   if (canvas_done) {
     if (valid && a.fmask) a.fmask[r] = 0;
   } else {
-    float e = valid ? __ldcg(&a.ent[r]) : INFINITY;
+    const int32_t draw = unf ? canvas_draw(seed, (uint32_t)(t + 1), (uint32_t)p, (uint32_t)b, (uint32_t)a.V) : 0;
     if (!(e == e)) e = INFINITY;  // NaN (already flagged) orders last
-    const bool unf = valid && a.frozen[r] == 0;
     // key = (entropy, position); frozen and padding slots sort after every unfrozen one
     const unsigned long long key =
         unf ? (((unsigned long long)float_order(e) << 32) | (unsigned)p) : ~0ull;
     const int U = __syncthreads_count(unf);
-    const int t = a.step[b];
     const int left = a.max_steps - t;
     const int k = (left <= 1) ? U : (U + left - 1) / left;
     const unsigned long long sorted = block_bitonic_sort(key, s_x);
@@ -183,7 +189,6 @@ __global__ void __launch_bounds__(kMaxSelect) merge_select_kernel(SelectArgs a) 
     if (p < k) s_freeze[(unsigned)(sorted & 0xffffffffu)] = 1;  // k <= U: an unfrozen position
     __syncthreads();
     const bool F = unf && s_freeze[p];
-    const int amv = valid ? __ldcg(&a.am[r]) : 0;
     if (F) {
       a.tok[r] = amv;
       a.frozen[r] = 1;
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(kMaxSelect) merge_select_kernel(SelectArgs a) 
       if (rest) a.tok[r] = amv;
       if (valid) a.frozen[r] = 1;
     } else if (rest) {
-      a.tok[r] = canvas_draw(a.seed[b], (uint32_t)(t + 1), (uint32_t)p, (uint32_t)b, (uint32_t)a.V);
+      a.tok[r] = draw;
     }
     if (valid && a.fmask) a.fmask[r] = F ? 1 : 0;
     if (threadIdx.x == 0) {

@@ -396,19 +396,27 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // completions arrive on both CTAs' stage-free and accumulator-full barriers;
 // all 16 epilogue warps of the pair arrive on the even CTA's accumulator-free
 // barrier.
-constexpr int kPairStages = 6;
+constexpr int kPairStages = 7;
 constexpr int kPairABytes = 128 * kRowBytes;                // 16 KB: this CTA's 128 rows
 constexpr int kPairBBytes = 128 * kRowBytes;                // 16 KB: up to 128 vocab rows
 constexpr int kPairStageBytes = kPairABytes + kPairBBytes;  // 32 KB
-constexpr int kPairMergeBytes = 128 * 32;                   // one row state per TMEM lane
-constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 1024 + 256 + kPairMergeBytes;
+// the dynamic shared window starts 1024-aligned (checked at entry): seven
+// 32 KB stages and the barriers fill it; the epilogue's merge area (one row
+// state per TMEM lane, 4 KB) reuses stage 0 once every MMA has completed
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 256;
 
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
   constexpr int kBK = kFp8 ? kRowBytes : kRowBytes / 2;  // K elements per block
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // SW128 tiles need 1024-byte alignment; the window's start is the same in
+  // both CTAs of the pair, so both return here (before any pair operation)
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) set_error(p.err, kDevBadAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;  // [2]
@@ -416,7 +424,7 @@ lmhead_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   uint64_t* mdone = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* merge_area = reinterpret_cast<float*>(smem + kPairStages * kPairStageBytes + 256);  // [128][8]
+  float* merge_area = reinterpret_cast<float*>(smem);  // [128][8], stage 0 after the last tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: the pair's MMA issuer
@@ -459,11 +467,8 @@ lmhead_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      const uint64_t polA = policy_evict_last();
-      // vocab rows: streamed once when one 256-row block reads them; with
-      // several blocks, the blocks' pairs read each row at slightly different
-      // times and the row should stay in L2 until the last of them
-      const uint64_t polB = gridDim.y > 1 ? policy_evict_normal() : policy_evict_first();
+      const uint64_t polA = policy_evict_last();   // rows' activations: re-read every tile
+      const uint64_t polB = policy_evict_first();  // vocab weights: streamed
       const uint32_t full_even = mapa_shared(full, 0);
       const uint32_t tx = 2 * kPairStageBytes;  // both CTAs' boxes (rows past M or V are zero-filled, counted)
       int s = 0;

@@ -327,6 +327,15 @@ def bench_reference(args, rank, world):
 FP8_OVER_BF16 = 2.0  # nominal dense ratio 4.5 / 2.25 PFLOP/s
 
 
+def peak_kind_of(region_s, clocks):
+    """Which measured tensor peak a kernel timed in the step loop is held to:
+    the sustained one (measured under the power cap) when the clock record of
+    the timed region shows the cap active, or the region lasted a second or
+    more; the burst one otherwise."""
+    capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
+    return "sustained" if (region_s >= SUSTAINED_AFTER_S or capped) else "burst"
+
+
 def kernel_roofline(name, kernel, flops, bytes_, avg_ms, peaks, peak_kind, traffic, fp8=False):
     """A contraction's roofline against the peak of its own operand type: the
     measured bf16 peak, times the nominal FP8/bf16 ratio for e4m3 operands."""
@@ -442,10 +451,7 @@ def bench_b200(args, rank, world, local_rank):
     for k in ev:
         cv.set_timing_events([], [], kernel=k)
     steps_per_s = job_rate(args.steps, world, elapsed_ms)
-    # the sustained peak is the one measured under the power cap: it applies
-    # when the timed kernels ran under it too, or ran a second or more
-    capped = "sw_power_cap" in (ck or {}).get("reasons", [])
-    peak_kind = "sustained" if (region2_s >= SUSTAINED_AFTER_S or capped) else "burst"
+    peak_kind = peak_kind_of(region2_s, ck)
     # more than 128 rows run on CTA pairs (lmhead_tc_pair_kernel)
     lm_kernel = "lmhead_tc_pair_kernel" if cfg.B * cfg.C > 128 else "lmhead_tc_kernel"
     lm = kernel_roofline("lmhead", lm_kernel + "<" + ("e4m3" if cfg.lm_fp8 else "bf16")

@@ -257,7 +257,7 @@ dg_status dg_canvas_set_state(dg_ctx *ctx, const dg_state *host_in);
  * dg_denoise_step without debug outputs records starts[i % n] just before and
  * stops[i % n] just after the kernel named by `kernel`: DG_KERNEL_LMHEAD (the
  * LM head with its entropy/argmax epilogue) or DG_KERNEL_ATTENTION (the
- * attention kernel, with its split-KV merge when it has one). n = 0 turns it
+ * attention kernel, with its merge kernel when CTAs share units). n = 0 turns it
  * off for that kernel; the settings are independent. DG_KERNEL_DECODE takes
  * one pair (n <= 1), recorded by dg_decode_block's graph just before its loop
  * starts and just after it ends (the device time of the loop alone); the

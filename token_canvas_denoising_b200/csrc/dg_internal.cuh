@@ -193,8 +193,9 @@ bool gemm_tc_prepare_with(GemmTc* g, const void* A, int M, int K, int nseg, cons
 size_t gemm_tc_partial_floats(const GemmTc& g);
 void launch_gemm_tc(Exec& ex, const GemmTc& g, const void* residual);
 
-// tcgen05 attention (bf16, head_dim 128): tensor maps per group of up to 8
-// requests, split-KV partial buffers.
+// tcgen05 attention (bf16, head_dim 128): tensor maps and the stream-K
+// schedule per group of up to 8 requests; partial buffers for the units that
+// several CTAs share.
 struct AttnTc {
   // stream-K schedule of one launch: the units' T key tiles over G CTAs, at
   // most `parts` CTAs per unit (the partial slots it needs)
